@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the Grok-1 MoE feed-forward layer on B200: tokens/s at the Grok-1
+shape (d_model 6144, ffn 32768, 8 experts, top-2, int8 weights) and the fraction
+of the HBM / bf16 tensor roofline reached by the dominant kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|stacked]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on the host cores
+
+One step = one pass of the whole layer (router, dispatch, gather, up-projection,
+down-projection, combine) over one batch of T synthetic tokens; the stacked
+workload's step is its four residual blocks.  Inputs are resident in HBM when
+the timed region starts; the layer weights (4.8 GB) are larger than L2, so every
+step streams them from HBM.  Under torchrun each rank runs an independent
+replica on its own GPU and its own token batch (no collective on the data path);
+the reported value is all ranks' tokens over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/sec at Grok-1 shape; % of HBM / bf16 tensor-pipe roofline"
+KERNELS = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=None)
+    p.add_argument("--warmup", type=int, default=None)
+    p.add_argument("--impl", choices=("native", "reference"), default="native")
+    p.add_argument("--workload", default="decode", choices=("decode", "prefill", "skewed", "stacked", "tiny"))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
+    return p.parse_args()
+
+
+def default_steps(workload):
+    # enough steps that the timed region lasts about a second or more
+    return {"decode": (1000, 20), "stacked": (300, 10), "prefill": (40, 5), "skewed": (60, 5),
+            "tiny": (1000, 20)}[workload]
+
+
+# ---- distributed plumbing --------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = os.environ.get("MOE_BENCH_BACKEND", "nccl")
+        if backend == "nccl":
+            import torch
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def dist_teardown(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---- clocks sampled during the timed region --------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.th = threading.Thread(target=self._read, daemon=True)
+        self.th.start()
+        t_end = time.time() + 5.0
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 and self.t1 and self.t0 <= r[0] <= self.t1]
+        use = inside if inside else rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = set()
+        for r in use:
+            for nm, v in zip(names, r[3][1:]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": sorted(reasons), "samples": len(use),
+                "window": "timed region" if inside else "whole run (timed region shorter than one sample)"}
+
+
+# ---- roofline bookkeeping ----------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "ptx.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "mixture_experts_softmax_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel has not changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(f"{workload}/{kernel}")
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def algorithmic_work(w, T, n_touched, counts):
+    """Per-launch algorithmic bytes and FLOPs of the up- and down-projection kernels."""
+    d, F = w.d, w.F
+    R = 2 * T
+    up_bytes = n_touched * (2 * d * F + 2 * 2 * F) + R * d * 2 + R * F * 2
+    dn_bytes = n_touched * (F * d + 2 * d) + R * F * 2 + R * d * 4
+    up_flops = 2.0 * R * d * F * 2
+    dn_flops = 2.0 * R * F * d
+    return dict(up_bytes=up_bytes, dn_bytes=dn_bytes, up_flops=up_flops, dn_flops=dn_flops)
+
+
+# ---- the CUDA path -------------------------------------------------------------------
+
+def run_native(args, world, rank, local):
+    import torch
+    import moe_synth
+    import mixture_experts_softmax_b200 as moe
+
+    w = moe_synth.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    K, W = args.steps, args.warmup
+    inp = moe_synth.make_inputs(w, device=dev, seed=w.seed)
+    if world > 1:   # each replica gets its own token batch; the layer weights are the same model
+        g = moe_synth.generator(w.seed + 1000 + rank, dev)
+        inp.x = moe_synth.draw_tokens(w.T, w.d, g, dev)
+    T = w.T
+    layers = inp.layers
+    bias = inp.bias
+    stream = torch.cuda.current_stream(dev)
+
+    h = moe.MoELayer(w.d, w.F, w.E, w.k)
+    moe.check(moe.moe_set_router_bias(h.h, bias))
+    out = torch.empty_like(inp.x)
+    res0 = inp.x.clone()
+
+    def step():
+        if w.blocks:
+            hio.copy_(res0)
+            for b in range(w.blocks):
+                moe.check(moe.moe_block_forward(h.h, T, hio, inp.gammas[b]["pre"], inp.gammas[b]["post"], w.eps,
+                                                *moe.layer_args(layers[b]), stream))
+        else:
+            moe.check(moe.moe_forward(h.h, T, inp.x, *moe.layer_args(layers[0]), out, stream))
+
+    hio = torch.empty_like(inp.x)
+    for _ in range(W):
+        step()
+    moe.check(moe.moe_sync_status(h.h, stream))
+
+    # headline: K steps, device-timed
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.mark("t0")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.mark("t1")
+    barrier(world, dev)
+    ms = e0.elapsed_time(e1) / K
+    clk = clocks.stop() if clocks else None
+    moe.check(moe.moe_sync_status(h.h, stream), "device status after the timed region")
+    ms_max = max_over_ranks(ms, world, dev)
+    tokens = T * world
+    value = tokens / (ms_max / 1e3)
+
+    # per-kernel durations: the same K steps again with events around every launch
+    moe.check(moe.moe_set_profiling(h.h, True))
+    moe.moe_get_kernel_times(h.h)
+    barrier(world, dev)
+    for _ in range(K):
+        step()
+    torch.cuda.synchronize(dev)
+    rc, ktimes = moe.moe_get_kernel_times(h.h)
+    moe.check(rc)
+    moe.check(moe.moe_set_profiling(h.h, False))
+    per_launch = {k: (t / n if n else 0.0) for k, (t, n) in ktimes.items()}
+    launches_per_step = sum(n for _, n in ktimes.values()) / K
+
+    # routing of the last step -> experts that received tokens
+    offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
+    moe.check(moe.moe_get_routing(h.h, None, None, offsets, None, stream))
+    off = offsets.cpu().tolist()
+    counts = [off[e + 1] - off[e] for e in range(w.E)]
+    n_touched = sum(1 for c in counts if c > 0)
+
+    # end to end through the host-buffer entry point (pinned host memory, copies timed)
+    e2e = None
+    if not w.blocks:
+        x_host = inp.x.cpu().pin_memory()
+        out_host = torch.empty_like(x_host).pin_memory()
+        for _ in range(max(1, W // 2)):
+            moe.check(moe.moe_forward_host(h.h, T, x_host, *moe.layer_args(layers[0]), out_host, stream))
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(K):
+            moe.check(moe.moe_forward_host(h.h, T, x_host, *moe.layer_args(layers[0]), out_host, stream))
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / K, world, dev)
+        moe.check(moe.moe_sync_status(h.h, stream))
+        nb = T * w.d * 2
+        e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": nb,
+               "d2h_bytes_per_step": nb, "ms_per_step": e2e_ms, "api": "moe_forward_host"}
+
+    peaks, peak_src = measured_peaks()
+    work = algorithmic_work(w, T, n_touched, counts)
+    up_ms = per_launch["up_proj"]
+    dn_ms = per_launch["down_proj"]
+    if args.workload in ("prefill", "skewed"):
+        achieved = work["up_flops"] / (up_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "kernel": "up_proj", "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "traffic": recorded_traffic(args.workload, "up_proj"),
+                "algorithmic_flops_per_launch": work["up_flops"], "launch_ms": up_ms}
+    else:
+        nb = work["up_bytes"] * (w.blocks or 1)
+        achieved = work["up_bytes"] / (up_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "kernel": "up_proj", "peak_source": f"{peak_src} hbm_gbs (copy)",
+                "traffic": recorded_traffic(args.workload, "up_proj"),
+                "algorithmic_bytes_per_launch": work["up_bytes"], "launch_ms": up_ms}
+        del nb
+    layer_bytes = (work["up_bytes"] + work["dn_bytes"]) * (w.blocks or 1)
+    layer_roof = {"bytes_per_step": layer_bytes, "GBps": layer_bytes / (ms / 1e3) / 1e9,
+                  "frac_hbm": layer_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                  "flops_per_step": (work["up_flops"] + work["dn_flops"]) * (w.blocks or 1)}
+    layer_roof["TFLOPs"] = layer_roof["flops_per_step"] / (ms / 1e3) / 1e12
+    layer_roof["frac_tensor"] = layer_roof["TFLOPs"] / peaks["bf16_tflops"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, layers, inp, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded; random-init int8 weights of the Grok-1 MoE shape)",
+        "config": {"workload": args.workload, "T_per_gpu": T, "d_model": w.d, "ffn": w.F, "experts": w.E,
+                   "top_k": w.k, "blocks": w.blocks or 1, "weights": "int8 + bf16 per-output-channel scales",
+                   "l2": "inputs larger than L2 (%.2f GB of weights per step)" % (layer_bytes / 1e9),
+                   "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],
+                   "down_splits": moe.moe_plan(h.h, T)[2]},
+        "roofline": roof,
+        "layer": layer_roof,
+        "kernel_ms": per_launch,
+        "experts_touched": n_touched,
+        "gpu_launches": int(round(launches_per_step * K)),
+        "e2e": e2e,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    h.close()
+    return line
+
+
+def cpu_baseline(w, layers, inp, budget_s):
+    """The fp64 oracle on the host cores on a bounded sample of the same workload."""
+    import numpy as np
+    import torch
+    import oracle
+    cpu_layers = [{k: v.cpu() for k, v in l.items()} for l in layers]
+    x = inp.x.cpu()
+    cores = os.cpu_count()
+    t_start = time.time()
+    done = 0
+    if w.blocks:
+        gam = [{k: v.cpu() for k, v in g.items()} for g in inp.gammas]
+        while done < x.shape[0] and (time.time() - t_start) < budget_s or done == 0:
+            oracle.block_chain(cpu_layers, gam, x, eps=w.eps, tokens=[done])
+            done += 1
+        sample = f"{done} of {x.shape[0]} tokens through all {w.blocks} blocks"
+    else:
+        bias = None if inp.bias is None else inp.bias.cpu()
+        oracle.route(x, cpu_layers[0]["router_w"], bias)   # routing of the whole batch
+        while done < x.shape[0] and (time.time() - t_start) < budget_s or done == 0:
+            oracle.forward(cpu_layers[0], x, bias=bias, tokens=[done])
+            done += 1
+        sample = f"routing of all {x.shape[0]} tokens + expert FFNs of {done} tokens"
+    dt = time.time() - t_start
+    return {"value": done / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+            "seconds": dt}
+
+
+# ---- the reference arm: the CPU oracle ------------------------------------------------
+
+def run_reference(args, world, rank):
+    import torch
+    import moe_synth
+    import oracle
+    w = moe_synth.WORKLOADS[args.workload]
+    inp = moe_synth.make_inputs(w, device="cpu")
+    K, W = args.steps, args.warmup
+    x = inp.x
+    bias = inp.bias
+    per_step_tokens = 1
+
+    def step(i):
+        t = i % x.shape[0]
+        if w.blocks:
+            oracle.block_chain(inp.layers, inp.gammas, x, eps=w.eps, tokens=[t])
+        else:
+            oracle.forward(inp.layers[0], x, bias=bias, tokens=[t])
+
+    for i in range(W):
+        step(i)
+    t0 = time.time()
+    for i in range(K):
+        step(W + i)
+    dt = time.time() - t0
+    value = K * per_step_tokens / dt
+    cores = os.cpu_count()
+    sample = f"{per_step_tokens} token of the {w.T}-token batch per step (expert FFNs of its 2 routes" + \
+             (f", all {w.blocks} blocks" if w.blocks else "") + ")"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": dt / K * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; random-init int8 weights of the Grok-1 MoE shape)",
+        "config": {"workload": args.workload, "T_per_gpu": w.T, "d_model": w.d, "ffn": w.F, "experts": w.E,
+                   "top_k": w.k, "blocks": w.blocks or 1},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    ks, ws = default_steps(args.workload)
+    if args.steps is None:
+        args.steps = ks
+    if args.warmup is None:
+        args.warmup = ws
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        if args.steps > 50 and args.workload != "tiny":
+            args.steps = 20    # each step is about a second of fp64 work on the host
+        line = run_reference(args, world, rank)
+        print(json.dumps(line), flush=True)
+        return 0
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        line = run_native(args, world, rank, local)
+    finally:
+        pass
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist_teardown(world)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

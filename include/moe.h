@@ -1,0 +1,190 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) Grok-1 mixture-of-experts feed-forward layer.
+ *
+ * The layer (as described in "Grok-1 Admin & Architecture Guide", section 3
+ * "The Model", "Mixture of Experts (MoELayer + Router)" and "Quantized weights"):
+ *
+ *   1. routing logits L = x . router_w in fp32, softmax over the E experts;
+ *   2. the top-2 experts of each token (ties go to the lower expert index);
+ *   3. each chosen expert e computes  y_e = linear_1( gelu(linear(x)) * linear_v(x) )
+ *      with 8-bit weights dequantised as  int8 value * per-output-channel bf16 scale;
+ *   4. out = p[e0] * y_e0 + p[e1] * y_e1, where p is the softmax probability
+ *      (the gates are not renormalised over the two picks).
+ * FFN width: "llm-architectures-explained: Grok-1", table "Every architecture
+ * field", row ffns.moe.d_expert (32768 at d_model 6144).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers unless the name ends in _host; the
+ *     caller owns all of them.  Every pointer must be 16-byte aligned and every
+ *     tensor dense and row-major with the layout stated below.
+ *   - bf16 tensors are passed as void* (IEEE bfloat16, 2 bytes per element).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls only enqueue work on it: none synchronises the host except
+ *     moe_sync_status and moe_get_kernel_times, which say so.
+ *   - Every call returns MOE_OK (0) or a negative MOE_E* code; no exception or
+ *     abort crosses the ABI.  Arguments are checked on the host before any CUDA
+ *     call, so an invalid call has no effect on the device.
+ *   - A handle is bound to the CUDA device that is current at its first
+ *     forward call.  Calls on one handle must not run concurrently from several
+ *     host threads (the handle's workspace is shared).
+ *
+ * Layout of one layer's parameters (E experts, model width d, FFN width F):
+ *   router_w  fp32 [d, E]      routing weight (x . router_w)
+ *   w_lin     int8 [E, d, F]   linear   (x @ W orientation), s_lin bf16 [E, F]
+ *   w_v       int8 [E, d, F]   linear_v,                     s_v   bf16 [E, F]
+ *   w_1       int8 [E, F, d]   linear_1,                     s_1   bf16 [E, d]
+ * Scales are per output channel:  W_deq[e, i, o] = w[e, i, o] * s[e, o].
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* ---- status codes ---------------------------------------------------------- */
+#define MOE_OK            0
+#define MOE_EINVAL       -1   /* invalid argument (null/misaligned pointer, bad size)      */
+#define MOE_EUNSUPPORTED -2   /* valid request this library does not implement           */
+#define MOE_ENOMEM       -3   /* device or host allocation failed                         */
+#define MOE_ECUDA        -4   /* a CUDA runtime call or kernel launch failed               */
+#define MOE_ETIMEOUT     -5   /* a bounded device-side wait ran out (see moe_sync_status)  */
+#define MOE_ENODEV       -6   /* no CUDA device, or not an sm_100 device                   */
+
+/* Largest token count one call accepts. */
+#define MOE_MAX_TOKENS   262144
+
+typedef struct moe_ctx *moe_handle;
+
+/* Human-readable text for a status code.  Never NULL; the string is static. */
+MOE_API const char *moe_strerror(int code);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+MOE_API int moe_version(void);
+
+/*
+ * Create a layer handle for model width d, FFN width ffn, E experts and k picks
+ * per token ("Configuration objects" of the admin guide: emb_size, the FFN
+ * width from widening_factor, num_experts, num_selected_experts).
+ * Supported: E == 8, k == 2, d % 128 == 0, ffn % 128 == 0, 128 <= d, ffn <= 65536.
+ * Returns MOE_EINVAL for non-positive sizes or k > E, MOE_EUNSUPPORTED for
+ * other shapes.  Allocates host memory only; device memory is taken on the
+ * first forward call (stream-ordered) and grows with the largest T seen.
+ * On success *out owns the handle; release it with moe_destroy.
+ */
+MOE_API int moe_create(int d, int ffn, int E, int k, moe_handle *out);
+
+/*
+ * Release the handle and its device workspace.  Waits for the handle's last
+ * enqueued work to finish first.  NULL is accepted and ignored.
+ */
+MOE_API int moe_destroy(moe_handle h);
+
+/*
+ * Add a fixed fp32 bias to every token's routing logits (after the fp32 dot
+ * product, before the softmax).  bias: device fp32 [E], or NULL to remove it.
+ * The pointer is kept, not copied: it must stay valid while forwards that use
+ * it run.  This is a test hook (the skewed-routing workload); the model itself
+ * has no router bias.
+ */
+MOE_API int moe_set_router_bias(moe_handle h, const float *bias);
+
+/*
+ * The MoE layer on T tokens ("Mixture of Experts (MoELayer + Router)", steps 1-4).
+ *   x    bf16 [T, d]   input tokens
+ *   out  bf16 [T, d]   output; must not overlap x or the weights
+ * Weights and scales as in the layout block above.  T == 0 is a no-op.
+ * Enqueues the router, dispatch, gather, up-projection, down-projection and
+ * combine kernels on `stream` and returns.  Deterministic: the same inputs give
+ * bit-identical outputs.  Device-side wait timeouts are reported later by
+ * moe_sync_status.  Returns MOE_EINVAL on a bad argument, MOE_ENOMEM if the
+ * workspace could not grow, MOE_ECUDA if a launch failed.
+ */
+MOE_API int moe_forward(moe_handle h, int T, const void *x, const float *router_w,
+                        const int8_t *w_lin, const void *s_lin, const int8_t *w_v,
+                        const void *s_v, const int8_t *w_1, const void *s_1, void *out,
+                        void *stream);
+
+/*
+ * moe_forward with the tokens and the result in HOST memory: copies x_host
+ * (bf16 [T, d]) to the device, runs the layer, copies the result into out_host
+ * (bf16 [T, d]), all enqueued on `stream`.  The weights are device pointers.
+ * Pinned host buffers make the copies asynchronous; the caller must
+ * synchronise the stream (e.g. moe_sync_status) before reading out_host.
+ */
+MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const float *router_w,
+                             const int8_t *w_lin, const void *s_lin, const int8_t *w_v,
+                             const void *s_v, const int8_t *w_1, const void *s_1,
+                             void *out_host, void *stream);
+
+/*
+ * One residual MoE block ("Transformer stack and language model head": pre/post
+ * RMSNorm around the MoE, h += h_dense), in place on the residual stream:
+ *   u = bf16( RMSNorm(h; g_pre) ),   h <- bf16( h + RMSNorm( MoE(u); g_post ) )
+ * with RMSNorm(z; g) = z / sqrt(mean(z^2) + eps) * g evaluated in fp32.
+ *   h_io          bf16 [T, d]  residual stream, read and overwritten
+ *   g_pre, g_post bf16 [d]     RMSNorm gains
+ * Other arguments as in moe_forward.
+ */
+MOE_API int moe_block_forward(moe_handle h, int T, void *h_io, const void *g_pre,
+                              const void *g_post, float eps, const float *router_w,
+                              const int8_t *w_lin, const void *s_lin, const int8_t *w_v,
+                              const void *s_v, const int8_t *w_1, const void *s_1, void *stream);
+
+/*
+ * Copy the routing of the handle's last forward (device to device, on `stream`):
+ *   idx     int32 [T, 2]  chosen experts, slot 0 = larger probability
+ *   gate    fp32  [T, 2]  their softmax probabilities
+ *   offsets int32 [E+1]   first row of each expert in the grouped order
+ *   perm    int32 [2T]    route id (2*t + slot) of each grouped row
+ * Any pointer may be NULL.  Returns MOE_EINVAL if no forward ran yet.
+ */
+MOE_API int moe_get_routing(moe_handle h, int32_t *idx, float *gate, int32_t *offsets,
+                            int32_t *perm, void *stream);
+
+/*
+ * Synchronise `stream`, then report the device status of the handle's kernels:
+ * MOE_OK, MOE_ETIMEOUT if a bounded wait inside a pipelined kernel ran out (the
+ * kernel then stopped early and its output is invalid), or MOE_ECUDA if the
+ * stream reported an error.  Reading the status clears it.
+ */
+MOE_API int moe_sync_status(moe_handle h, void *stream);
+
+/*
+ * Limit, in nanoseconds, of every bounded wait inside the pipelined GEMM
+ * kernels (default 2e9).  A wait that runs out records MOE_ETIMEOUT and the
+ * kernel returns early with its async copies drained.  0 makes any wait that
+ * does not succeed at once give up: a test hook for the timeout path.
+ */
+MOE_API int moe_set_timeout(moe_handle h, long long ns);
+
+/*
+ * Per-kernel timing with CUDA events recorded on the launch stream.
+ * moe_set_profiling(h, 1) starts recording around each kernel of every forward;
+ * moe_get_kernel_times synchronises on those events and returns, per kernel id
+ * (0 router, 1 dispatch, 2 gather, 3 up-projection, 4 down-projection,
+ * 5 combine, 6 pre-norm), the total milliseconds and the launch count since the
+ * previous call, then resets them.  n = capacity of ms/launches (7 suffices).
+ */
+MOE_API int moe_set_profiling(moe_handle h, int on);
+MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
+
+/*
+ * The tile shape and split chosen for T tokens (for tests and benchmarks):
+ * *bn = routes per GEMM tile, *splits = K-splits of the down-projection.
+ */
+MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,215 @@
+"""Grok-1 mixture-of-experts feed-forward layer on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libmoe_b200.so``, whose C ABI is declared in
+``include/moe.h``.  Each function here has the name of its C entry point and
+only marshals arguments: tensors become device (or host) pointers, the stream
+becomes a ``cudaStream_t``.  Every step of the layer runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback, and importing this package
+fails loudly if the library has not been built.
+
+Functions return the library's integer status (``MOE_OK`` = 0); ``check`` turns
+a non-zero status into ``MoEError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_EINVAL = -1
+MOE_EUNSUPPORTED = -2
+MOE_ENOMEM = -3
+MOE_ECUDA = -4
+MOE_ETIMEOUT = -5
+MOE_ENODEV = -6
+MOE_MAX_TOKENS = 262144
+
+KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm")
+
+# every symbol include/moe.h declares
+EXPORTS = (
+    "moe_strerror", "moe_version", "moe_create", "moe_destroy", "moe_set_router_bias",
+    "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing",
+    "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
+)
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {moe_strerror(code)} ({code})" if what else f"{moe_strerror(code)} ({code})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m mixture_experts_softmax_b200.build` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sig = {
+        "moe_strerror": (ctypes.c_char_p, [I]),
+        "moe_version": (I, []),
+        "moe_create": (I, [I, I, I, I, ctypes.POINTER(P)]),
+        "moe_destroy": (I, [P]),
+        "moe_set_router_bias": (I, [P, P]),
+        "moe_forward": (I, [P, I, P, P, P, P, P, P, P, P, P, P]),
+        "moe_forward_host": (I, [P, I, P, P, P, P, P, P, P, P, P, P]),
+        "moe_block_forward": (I, [P, I, P, P, P, F, P, P, P, P, P, P, P, P]),
+        "moe_get_routing": (I, [P, P, P, P, P, P]),
+        "moe_sync_status": (I, [P, P]),
+        "moe_set_timeout": (I, [P, ctypes.c_longlong]),
+        "moe_set_profiling": (I, [P, I]),
+        "moe_get_kernel_times": (I, [P, P, P, I]),
+        "moe_plan": (I, [P, I, ctypes.POINTER(I), ctypes.POINTER(I)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _ptr(t) -> Optional[int]:
+    """torch tensor / int / None -> raw address."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        return t.data_ptr()
+    raise TypeError(f"cannot pass {type(t).__name__} as a pointer")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def check(rc: int, what: str = "") -> None:
+    if rc != MOE_OK:
+        raise MoEError(rc, what)
+
+
+def moe_strerror(code: int) -> str:
+    return _lib.moe_strerror(int(code)).decode()
+
+
+def moe_version() -> int:
+    return _lib.moe_version()
+
+
+def moe_create(d: int, ffn: int, E: int = 8, k: int = 2) -> Tuple[int, Optional[int]]:
+    h = ctypes.c_void_p()
+    rc = _lib.moe_create(d, ffn, E, k, ctypes.byref(h))
+    return rc, h.value
+
+
+def moe_destroy(h) -> int:
+    return _lib.moe_destroy(h)
+
+
+def moe_set_router_bias(h, bias) -> int:
+    return _lib.moe_set_router_bias(h, _ptr(bias))
+
+
+def moe_forward(h, T, x, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, out, stream=None) -> int:
+    return _lib.moe_forward(h, int(T), _ptr(x), _ptr(router_w), _ptr(w_lin), _ptr(s_lin), _ptr(w_v),
+                            _ptr(s_v), _ptr(w_1), _ptr(s_1), _ptr(out), _stream(stream))
+
+
+def moe_forward_host(h, T, x_host, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, out_host, stream=None) -> int:
+    return _lib.moe_forward_host(h, int(T), _ptr(x_host), _ptr(router_w), _ptr(w_lin), _ptr(s_lin),
+                                 _ptr(w_v), _ptr(s_v), _ptr(w_1), _ptr(s_1), _ptr(out_host), _stream(stream))
+
+
+def moe_block_forward(h, T, h_io, g_pre, g_post, eps, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1,
+                      stream=None) -> int:
+    return _lib.moe_block_forward(h, int(T), _ptr(h_io), _ptr(g_pre), _ptr(g_post), float(eps),
+                                  _ptr(router_w), _ptr(w_lin), _ptr(s_lin), _ptr(w_v), _ptr(s_v),
+                                  _ptr(w_1), _ptr(s_1), _stream(stream))
+
+
+def moe_get_routing(h, idx=None, gate=None, offsets=None, perm=None, stream=None) -> int:
+    return _lib.moe_get_routing(h, _ptr(idx), _ptr(gate), _ptr(offsets), _ptr(perm), _stream(stream))
+
+
+def moe_sync_status(h, stream=None) -> int:
+    return _lib.moe_sync_status(h, _stream(stream))
+
+
+def moe_set_timeout(h, ns: int) -> int:
+    return _lib.moe_set_timeout(h, int(ns))
+
+
+def moe_set_profiling(h, on: bool) -> int:
+    return _lib.moe_set_profiling(h, 1 if on else 0)
+
+
+def moe_get_kernel_times(h):
+    """-> (status, {kernel name: (total ms, launches)}) since the previous call."""
+    n = len(KERNEL_NAMES)
+    ms = (ctypes.c_float * n)()
+    cnt = (ctypes.c_int * n)()
+    rc = _lib.moe_get_kernel_times(h, ms, cnt, n)
+    return rc, {KERNEL_NAMES[i]: (ms[i], cnt[i]) for i in range(n)}
+
+
+def moe_plan(h, T: int):
+    """-> (status, routes per GEMM tile, K-splits of the down-projection) for T tokens."""
+    bn, sp = ctypes.c_int(), ctypes.c_int()
+    rc = _lib.moe_plan(h, int(T), ctypes.byref(bn), ctypes.byref(sp))
+    return rc, bn.value, sp.value
+
+
+def layer_args(layer: dict):
+    """The weight arguments of moe_forward, in order, from a dict with keys
+    router_w, wl, sl, wv, sv, w1, s1."""
+    return (layer["router_w"], layer["wl"], layer["sl"], layer["wv"], layer["sv"], layer["w1"], layer["s1"])
+
+
+class MoELayer:
+    """Owns one handle; raises MoEError on any non-zero status."""
+
+    def __init__(self, d: int, ffn: int, E: int = 8, k: int = 2):
+        rc, self.h = moe_create(d, ffn, E, k)
+        check(rc, "moe_create")
+        self.d, self.ffn, self.E, self.k = d, ffn, E, k
+
+    def close(self):
+        if self.h:
+            moe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def forward(self, x, layer: dict, out, stream=None):
+        check(moe_forward(self.h, x.shape[0], x, *layer_args(layer), out, stream), "moe_forward")
+        return out
+
+    def block_forward(self, h_io, g_pre, g_post, eps, layer: dict, stream=None):
+        check(moe_block_forward(self.h, h_io.shape[0], h_io, g_pre, g_post, eps, *layer_args(layer), stream),
+              "moe_block_forward")
+        return h_io
+
+    def sync(self, stream=None):
+        check(moe_sync_status(self.h, stream), "moe_sync_status")

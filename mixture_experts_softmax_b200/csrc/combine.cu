@@ -1,0 +1,100 @@
+// combine.cu -- sum the gate-weighted expert outputs back in token order
+// ("Grok-1 Admin & Architecture Guide", section 3, "Mixture of Experts", step 4),
+// and the residual-block variant with the post-MoE RMSNorm and residual add
+// ("Transformer stack and language model head": h += h_dense).
+//
+// The down-projection epilogue has already written gate * s1 * (partial sum) of
+// every route into its own slot [split, t, j, :].  Here each output element is the
+// sum of its 2 * splits slots in a fixed order (split ascending, slot 0 before
+// slot 1), so the result does not depend on scheduling.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ float4 ld4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+
+__device__ __forceinline__ void add4(float4 &a, const float4 &b)
+{
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+}
+
+// fixed-order sum of one token's slots for 4 consecutive features
+__device__ __forceinline__ float4 slot_sum(const CombineArgs &a, int t, int c)
+{
+    const size_t plane = static_cast<size_t>(a.T) * 2 * a.d;
+    const float *p = a.slots + (static_cast<size_t>(t) * 2) * a.d + c;
+    float4 y0 = ld4(p), y1 = ld4(p + a.d);
+    for (int s = 1; s < a.splits; ++s) {
+        add4(y0, ld4(p + s * plane));
+        add4(y1, ld4(p + s * plane + a.d));
+    }
+    add4(y0, y1);
+    return y0;
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
+{
+    const int per_row = a.d >> 2;
+    const size_t n = static_cast<size_t>(a.T) * per_row;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const int t = static_cast<int>(i / per_row), c = static_cast<int>(i % per_row) * 4;
+        const float4 y = slot_sum(a, t, c);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(y.x, y.y), hi = __floats2bfloat162_rn(y.z, y.w);
+        uint2 v;
+        v.x = *reinterpret_cast<uint32_t *>(&lo);
+        v.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(a.out + static_cast<size_t>(t) * a.d + c) = v;
+    }
+}
+
+// one block per token: y = sum of slots; h <- bf16( h + y * rsqrt(mean(y^2) + eps) * g_post )
+__global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
+{
+    __shared__ float red[8];
+    const int t = blockIdx.x;
+    float ss = 0.f;
+    for (int c = threadIdx.x * 4; c < a.d; c += blockDim.x * 4) {
+        const float4 y = slot_sum(a, t, c);
+        ss = fmaf(y.x, y.x, fmaf(y.y, y.y, fmaf(y.z, y.z, fmaf(y.w, y.w, ss))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const float r = rsqrtf(tot / static_cast<float>(a.d) + a.eps);
+    __nv_bfloat16 *hr = a.h_io + static_cast<size_t>(t) * a.d;
+    for (int c = threadIdx.x * 4; c < a.d; c += blockDim.x * 4) {
+        const float4 y = slot_sum(a, t, c);
+        const float yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float hv = __bfloat162float(hr[c + q]);
+            hr[c + q] = __float2bfloat16_rn(hv + yv[q] * r * __bfloat162float(a.g_post[c + q]));
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s)
+{
+    if (a.T <= 0) return cudaSuccess;
+    if (a.h_io) {
+        combine_postnorm_kernel<<<a.T, 256, 0, s>>>(a);
+    } else {
+        const size_t n = static_cast<size_t>(a.T) * (a.d >> 2);
+        const size_t want = (n + 255) / 256;
+        const int grid = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+        combine_kernel<<<grid, 256, 0, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

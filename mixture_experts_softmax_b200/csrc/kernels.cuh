@@ -1,0 +1,101 @@
+// kernels.cuh -- launch interface between the C ABI (moe_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kExperts = 8;       // E supported by the router kernel
+constexpr int kTopK = 2;          // picks per token
+constexpr int kBM = 128;          // output features per GEMM tile (TMEM lanes)
+constexpr int kBK = 64;           // reduction elements per pipeline stage (128 B of bf16)
+constexpr int kMaxSplits = 8;     // K-splits of the down-projection
+
+// device error word values (the first error wins)
+constexpr int kErrTimeoutBase = 0x1000;   // + wait site
+
+struct RouteArgs {
+    int T, d;
+    const __nv_bfloat16 *x;     // [T, d]
+    const float *w;             // [d, E]
+    const float *bias;          // [E] or nullptr
+    int *idx;                   // [T, 2]
+    float *gate;                // [T, 2]
+};
+
+struct DispatchArgs {
+    int T, E, bn;
+    const int *idx;             // [T, 2]
+    int *counts;                // [E]
+    int *offsets;               // [E+1]   unpadded grouped offsets
+    int *poff;                  // [E+1]   offsets with each expert's segment padded to bn rows
+    int *perm;                  // [2T]    grouped row -> route id (2t + slot)
+    int *rperm;                 // [rows]  padded row -> route id, -1 for padding
+    int *slot_of_route;         // [2T]    route id -> padded row
+};
+
+struct GatherArgs {
+    int d, max_rows;
+    const int *poff_end;        // &poff[E]: number of padded rows (device)
+    const int *rperm;
+    const __nv_bfloat16 *x;     // [T, d]
+    __nv_bfloat16 *xp;          // [rows, d]
+};
+
+// one grouped GEMM of the layer:  for every expert e and padded row r of e
+//   UP   (two A matrices):  H[r, f]  = bf16( gelu(s0[e,f] * A0) * (s1[e,f] * A1) )
+//   DOWN (one A matrix):    slot[s, t, j, f] = gate[t, j] * s0[e, f] * A0_partial(s)
+// where A_i[f, r] = sum_k W_i[e, k, f] * B[r, k] over this split's k range.
+struct GemmArgs {
+    int T;                      // tokens
+    int E;
+    int M;                      // output features (F for UP, d for DOWN)
+    int K;                      // reduction length (d for UP, F for DOWN)
+    int ksteps;                 // k-steps of kBK per split
+    int splits;                 // K-splits (DOWN); 1 for UP
+    const int *poff;            // [E+1]
+    const int *rperm;           // [rows]
+    const float *gate;          // [T, 2]
+    const __nv_bfloat16 *s0;    // [E, M]
+    const __nv_bfloat16 *s1;    // [E, M] (UP only)
+    __nv_bfloat16 *h;           // UP output   [rows, M]
+    float *slots;               // DOWN output [splits, T, 2, M]
+    int *err;                   // device error word
+    long long timeout_ns;
+};
+
+struct CombineArgs {
+    int T, d, splits;
+    const float *slots;         // [splits, T, 2, d]
+    __nv_bfloat16 *out;         // [T, d]
+    // residual block variant
+    __nv_bfloat16 *h_io;        // [T, d] residual stream (nullptr: plain combine)
+    const __nv_bfloat16 *g_post;
+    float eps;
+};
+
+struct NormArgs {
+    int T, d;
+    const __nv_bfloat16 *h;     // [T, d]
+    const __nv_bfloat16 *g;     // [d]
+    float eps;
+    __nv_bfloat16 *u;           // [T, d]
+};
+
+cudaError_t launch_router(const RouteArgs &a, cudaStream_t s);
+cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
+cudaError_t launch_gather(const GatherArgs &a, cudaStream_t s);
+cudaError_t launch_gemm_up(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
+                           const GemmArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_down(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,
+                             int grid, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+cudaError_t launch_prenorm(const NormArgs &a, cudaStream_t s);
+
+// dynamic shared memory each GEMM variant needs (for cudaFuncSetAttribute)
+size_t gemm_smem_bytes(bool up, int bn);
+
+}  // namespace moe

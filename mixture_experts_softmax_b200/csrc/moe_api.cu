@@ -1,0 +1,600 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: handle, argument checks,
+// workspace, TMA descriptors and the launch sequence of one MoE layer.
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+enum KernelId { K_ROUTER = 0, K_DISPATCH, K_GATHER, K_UP, K_DOWN, K_COMBINE, K_PRENORM };
+
+struct DevBuf {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+
+struct WeightMap {
+    const void *ptr = nullptr;
+    int kind = -1;   // 0: [E*d, F] (linear, linear_v)   1: [E*F, d] (linear_1)
+    CUtensorMap map;
+};
+
+struct PendingEvent {
+    int id;
+    cudaEvent_t a, b;
+};
+
+}  // namespace
+
+struct moe_ctx {
+    int d, F, E, k;
+    int device = -1;
+    int num_sms = 0;
+    cudaStream_t last_stream = nullptr;
+    bool used = false;
+
+    // workspace
+    DevBuf b_route;    // idx [2T] int, gate [2T] float, counts/offsets/poff, perm [2T], slot_of_route [2T]
+    DevBuf b_rperm;    // [rows]
+    DevBuf b_xp;       // bf16 [rows, d]
+    DevBuf b_h;        // bf16 [rows, F]
+    DevBuf b_slots;    // fp32 [splits, T, 2, d]
+    DevBuf b_stage;    // bf16 [T, d] x2: host-API input/output staging, block pre-norm output
+    int *err = nullptr;
+    int rows_cap = 0;       // rows the xp / h buffers hold
+    int route_cap = 0;      // T the route buffer holds
+    int map_gen = 0;        // bumps when b_xp / b_h move
+    int last_T = -1;
+
+    // TMA descriptors
+    std::vector<WeightMap> wmaps;
+    CUtensorMap xp_map[4], h_map[4];
+    int xp_map_gen[4] = {-1, -1, -1, -1}, h_map_gen[4] = {-1, -1, -1, -1};
+
+    const float *bias = nullptr;
+    long long timeout_ns = 2000000000LL;
+
+    // profiling
+    bool prof = false;
+    std::vector<PendingEvent> pending;
+    std::vector<cudaEvent_t> event_pool;
+};
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int plan_bn(int T)
+{
+    if (T <= 16) return 16;
+    if (T <= 32) return 32;
+    if (T <= 64) return 64;
+    return 128;
+}
+
+int bn_slot(int bn) { return bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3; }
+
+int plan_splits(const moe_ctx *h, int T, int bn)
+{
+    const int per_expert = (2 * T + h->E - 1) / h->E;
+    const long nt = per_expert <= bn ? 1 : (per_expert + bn - 1) / bn;
+    const long tiles = static_cast<long>(h->E) * (h->d / kBM) * nt;
+    const int ksteps = h->F / kBK;
+    const int sms = h->num_sms > 0 ? h->num_sms : 148;
+    int s = 1;
+    while (s < kMaxSplits && tiles * s < 16L * sms && ksteps % (2 * s) == 0) s *= 2;
+    return s;
+}
+
+int rows_for(const moe_ctx *h, int T, int bn) { return ((2 * T + h->E * (bn - 1)) + 127) / 128 * 128; }
+
+// route buffer layout (ints/floats), all offsets in 4-byte words
+struct RouteLayout {
+    size_t idx, gate, counts, offsets, poff, perm, slot, words;
+};
+
+RouteLayout route_layout(int T, int E)
+{
+    auto up = [](size_t v) { return (v + 63) / 64 * 64; };
+    RouteLayout L;
+    size_t o = 0;
+    L.idx = o; o += up(2 * static_cast<size_t>(T));
+    L.gate = o; o += up(2 * static_cast<size_t>(T));
+    L.counts = o; o += up(E);
+    L.offsets = o; o += up(E + 1);
+    L.poff = o; o += up(E + 1);
+    L.perm = o; o += up(2 * static_cast<size_t>(T));
+    L.slot = o; o += up(2 * static_cast<size_t>(T));
+    L.words = o;
+    return L;
+}
+
+int sync_last(moe_ctx *h)
+{
+    if (!h->used) return MOE_OK;
+    return cudaStreamSynchronize(h->last_stream) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+// grow a buffer to at least `bytes` (contents are not kept)
+int ensure(moe_ctx *h, DevBuf &b, size_t bytes, bool *moved = nullptr)
+{
+    if (b.bytes >= bytes) return MOE_OK;
+    if (b.ptr) {
+        if (sync_last(h) != MOE_OK) return MOE_ECUDA;
+        cudaFree(b.ptr);
+        b.ptr = nullptr;
+        b.bytes = 0;
+    }
+    size_t want = bytes + bytes / 4;   // headroom against repeated small growth
+    if (cudaMalloc(&b.ptr, want) != cudaSuccess) {
+        cudaGetLastError();
+        b.ptr = nullptr;
+        if (cudaMalloc(&b.ptr, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            b.ptr = nullptr;
+            return MOE_ENOMEM;
+        }
+        want = bytes;
+    }
+    b.bytes = want;
+    if (moved) *moved = true;
+    return MOE_OK;
+}
+
+int ensure_device(moe_ctx *h)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ENODEV;
+    }
+    if (h->device < 0) {
+        cudaDeviceProp p;
+        if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ENODEV;
+        }
+        if (p.major != 10) return MOE_ENODEV;   // built for sm_100a only
+        h->device = dev;
+        h->num_sms = p.multiProcessorCount;
+        if (cudaMalloc(reinterpret_cast<void **>(&h->err), 256) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ENOMEM;
+        }
+        if (cudaMemset(h->err, 0, 256) != cudaSuccess) return MOE_ECUDA;
+    } else if (dev != h->device) {
+        return MOE_EINVAL;   // the handle belongs to another device
+    }
+    return MOE_OK;
+}
+
+int ensure_workspace(moe_ctx *h, int T, int bn, int splits)
+{
+    int rc;
+    const RouteLayout L = route_layout(T, h->E);
+    if ((rc = ensure(h, h->b_route, L.words * 4)) != MOE_OK) return rc;
+    const int rows = rows_for(h, T, bn);
+    bool moved = false;
+    if (rows > h->rows_cap) {
+        if ((rc = ensure(h, h->b_rperm, static_cast<size_t>(rows) * 4)) != MOE_OK) return rc;
+        if ((rc = ensure(h, h->b_xp, static_cast<size_t>(rows) * h->d * 2, &moved)) != MOE_OK) return rc;
+        if ((rc = ensure(h, h->b_h, static_cast<size_t>(rows) * h->F * 2, &moved)) != MOE_OK) return rc;
+        h->rows_cap = rows;
+        // the descriptors cover rows_cap rows: rebuild them all
+        h->map_gen++;
+    }
+    (void)moved;
+    if ((rc = ensure(h, h->b_slots, static_cast<size_t>(splits) * T * 2 * h->d * 4)) != MOE_OK) return rc;
+    if ((rc = ensure(h, h->b_stage, static_cast<size_t>(T) * h->d * 2 * 2)) != MOE_OK) return rc;
+    return MOE_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D tiled map with 128-byte swizzle: inner extent `cols` elements, `rows` rows
+int encode_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *ptr, uint64_t cols, uint64_t rows,
+              uint32_t box_cols, uint32_t box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return MOE_ECUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ECUDA;
+}
+
+int weight_map(moe_ctx *h, const void *ptr, int kind, const CUtensorMap **out)
+{
+    for (auto &w : h->wmaps)
+        if (w.ptr == ptr && w.kind == kind) {
+            *out = &w.map;
+            return MOE_OK;
+        }
+    WeightMap w;
+    w.ptr = ptr;
+    w.kind = kind;
+    const uint64_t rows = kind == 0 ? static_cast<uint64_t>(h->E) * h->d : static_cast<uint64_t>(h->E) * h->F;
+    const uint64_t cols = kind == 0 ? h->F : h->d;
+    int rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, cols, rows, kBM, kBK);
+    if (rc != MOE_OK) return rc;
+    if (h->wmaps.size() >= 64) h->wmaps.erase(h->wmaps.begin());
+    h->wmaps.push_back(w);
+    *out = &h->wmaps.back().map;
+    return MOE_OK;
+}
+
+int act_maps(moe_ctx *h, int bn, const CUtensorMap **xp, const CUtensorMap **hm)
+{
+    const int s = bn_slot(bn);
+    int rc;
+    if (h->xp_map_gen[s] != h->map_gen) {
+        if ((rc = encode_2d(&h->xp_map[s], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->b_xp.ptr, h->d, h->rows_cap, kBK,
+                            bn)) != MOE_OK)
+            return rc;
+        h->xp_map_gen[s] = h->map_gen;
+    }
+    if (h->h_map_gen[s] != h->map_gen) {
+        if ((rc = encode_2d(&h->h_map[s], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->b_h.ptr, h->F, h->rows_cap, kBK,
+                            bn)) != MOE_OK)
+            return rc;
+        h->h_map_gen[s] = h->map_gen;
+    }
+    *xp = &h->xp_map[s];
+    *hm = &h->h_map[s];
+    return MOE_OK;
+}
+
+cudaEvent_t take_event(moe_ctx *h)
+{
+    if (!h->event_pool.empty()) {
+        cudaEvent_t e = h->event_pool.back();
+        h->event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return e;
+}
+
+// run one launch, bracketed by events when profiling
+template <class F>
+cudaError_t timed(moe_ctx *h, int id, cudaStream_t s, F &&launch)
+{
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (h->prof) {
+        a = take_event(h);
+        b = take_event(h);
+        if (a) cudaEventRecord(a, s);
+    }
+    cudaError_t e = launch();
+    if (h->prof && a && b) {
+        cudaEventRecord(b, s);
+        h->pending.push_back({id, a, b});
+    }
+    return e;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+int check_weights(const moe_ctx *h, const float *router_w, const int8_t *w_lin, const void *s_lin, const int8_t *w_v,
+                  const void *s_v, const int8_t *w_1, const void *s_1)
+{
+    const void *ps[] = {router_w, w_lin, s_lin, w_v, s_v, w_1, s_1};
+    for (const void *p : ps)
+        if (!p || !aligned16(p)) return MOE_EINVAL;
+    (void)h;
+    return MOE_OK;
+}
+
+// the layer on x (device, bf16 [T, d]); result into `out` (plain) or added into h_io (residual block)
+int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int8_t *w_lin, const void *s_lin,
+              const int8_t *w_v, const void *s_v, const int8_t *w_1, const void *s_1, void *out, void *h_io,
+              const void *g_post, float eps, cudaStream_t s)
+{
+    int rc;
+    const int bn = plan_bn(T);
+    const int splits = plan_splits(h, T, bn);
+    const RouteLayout L = route_layout(T, h->E);
+    int *rw = static_cast<int *>(h->b_route.ptr);
+    int *idx = rw + L.idx;
+    float *gate = reinterpret_cast<float *>(rw + L.gate);
+    int *poff = rw + L.poff;
+    int *rperm = static_cast<int *>(h->b_rperm.ptr);
+    const int rows = rows_for(h, T, bn);
+
+    const CUtensorMap *m_wl, *m_wv, *m_w1, *m_xp, *m_h;
+    if ((rc = weight_map(h, w_lin, 0, &m_wl)) != MOE_OK) return rc;
+    if ((rc = weight_map(h, w_v, 0, &m_wv)) != MOE_OK) return rc;
+    if ((rc = weight_map(h, w_1, 1, &m_w1)) != MOE_OK) return rc;
+    if ((rc = act_maps(h, bn, &m_xp, &m_h)) != MOE_OK) return rc;
+
+    RouteArgs ra{T, h->d, static_cast<const __nv_bfloat16 *>(x), router_w, h->bias, idx, gate};
+    if (timed(h, K_ROUTER, s, [&] { return launch_router(ra, s); }) != cudaSuccess) return MOE_ECUDA;
+
+    DispatchArgs da{T, h->E, bn, idx, rw + L.counts, rw + L.offsets, poff, rw + L.perm, rperm, rw + L.slot};
+    if (timed(h, K_DISPATCH, s, [&] { return launch_dispatch(da, s); }) != cudaSuccess) return MOE_ECUDA;
+
+    GatherArgs ga{h->d, rows, poff + h->E, rperm, static_cast<const __nv_bfloat16 *>(x),
+                  static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
+    if (timed(h, K_GATHER, s, [&] { return launch_gather(ga, s); }) != cudaSuccess) return MOE_ECUDA;
+
+    GemmArgs up{};
+    up.T = T;
+    up.E = h->E;
+    up.M = h->F;
+    up.K = h->d;
+    up.ksteps = h->d / kBK;
+    up.splits = 1;
+    up.poff = poff;
+    up.rperm = rperm;
+    up.gate = gate;
+    up.s0 = static_cast<const __nv_bfloat16 *>(s_lin);
+    up.s1 = static_cast<const __nv_bfloat16 *>(s_v);
+    up.h = static_cast<__nv_bfloat16 *>(h->b_h.ptr);
+    up.err = h->err;
+    up.timeout_ns = h->timeout_ns;
+    if (timed(h, K_UP, s, [&] { return launch_gemm_up(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s); }) != cudaSuccess)
+        return MOE_ECUDA;
+
+    GemmArgs dn = up;
+    dn.M = h->d;
+    dn.K = h->F;
+    dn.splits = splits;
+    dn.ksteps = h->F / kBK / splits;
+    dn.s0 = static_cast<const __nv_bfloat16 *>(s_1);
+    dn.s1 = nullptr;
+    dn.h = nullptr;
+    dn.slots = static_cast<float *>(h->b_slots.ptr);
+    if (timed(h, K_DOWN, s, [&] { return launch_gemm_down(bn, *m_w1, *m_h, dn, h->num_sms, s); }) != cudaSuccess)
+        return MOE_ECUDA;
+
+    CombineArgs ca{T, h->d, splits, static_cast<const float *>(h->b_slots.ptr), static_cast<__nv_bfloat16 *>(out),
+                   static_cast<__nv_bfloat16 *>(h_io), static_cast<const __nv_bfloat16 *>(g_post), eps};
+    if (timed(h, K_COMBINE, s, [&] { return launch_combine(ca, s); }) != cudaSuccess) return MOE_ECUDA;
+    h->last_T = T;
+    return MOE_OK;
+}
+
+int begin_call(moe_ctx *h, int T, cudaStream_t s)
+{
+    int rc;
+    if ((rc = ensure_device(h)) != MOE_OK) return rc;
+    if (h->used && s != h->last_stream) {
+        // work of the previous stream may still use the workspace
+        if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
+    }
+    const int bn = plan_bn(T);
+    if ((rc = ensure_workspace(h, T, bn, plan_splits(h, T, bn))) != MOE_OK) return rc;
+    h->last_stream = s;
+    h->used = true;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API const char *moe_strerror(int code)
+{
+    switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_EINVAL: return "invalid argument";
+    case MOE_EUNSUPPORTED: return "unsupported shape or option";
+    case MOE_ENOMEM: return "out of device memory";
+    case MOE_ECUDA: return "CUDA error";
+    case MOE_ETIMEOUT: return "device-side wait timed out";
+    case MOE_ENODEV: return "no sm_100 CUDA device";
+    default: return "unknown status code";
+    }
+}
+
+MOE_API int moe_version(void) { return 100; }
+
+MOE_API int moe_create(int d, int ffn, int E, int k, moe_handle *out)
+{
+    if (!out) return MOE_EINVAL;
+    *out = nullptr;
+    if (d <= 0 || ffn <= 0 || E <= 0 || k <= 0 || k > E) return MOE_EINVAL;
+    if (E != kExperts || k != kTopK) return MOE_EUNSUPPORTED;
+    if (d % kBM || ffn % kBM || d < kBM || ffn < kBM || d > 65536 || ffn > 65536) return MOE_EUNSUPPORTED;
+    moe_ctx *h = new (std::nothrow) moe_ctx();
+    if (!h) return MOE_ENOMEM;
+    h->d = d;
+    h->F = ffn;
+    h->E = E;
+    h->k = k;
+    *out = h;
+    return MOE_OK;
+}
+
+MOE_API int moe_destroy(moe_handle h)
+{
+    if (!h) return MOE_OK;
+    sync_last(h);
+    for (DevBuf *b : {&h->b_route, &h->b_rperm, &h->b_xp, &h->b_h, &h->b_slots, &h->b_stage})
+        if (b->ptr) cudaFree(b->ptr);
+    if (h->err) cudaFree(h->err);
+    for (auto &p : h->pending) {
+        cudaEventDestroy(p.a);
+        cudaEventDestroy(p.b);
+    }
+    for (auto e : h->event_pool) cudaEventDestroy(e);
+    delete h;
+    return MOE_OK;
+}
+
+MOE_API int moe_set_router_bias(moe_handle h, const float *bias)
+{
+    if (!h) return MOE_EINVAL;
+    if (bias && !aligned16(bias)) return MOE_EINVAL;
+    h->bias = bias;
+    return MOE_OK;
+}
+
+MOE_API int moe_set_timeout(moe_handle h, long long ns)
+{
+    if (!h || ns < 0) return MOE_EINVAL;
+    h->timeout_ns = ns;
+    return MOE_OK;
+}
+
+MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits)
+{
+    if (!h || T < 0 || T > MOE_MAX_TOKENS) return MOE_EINVAL;
+    const int b = plan_bn(T);
+    if (bn) *bn = b;
+    if (splits) *splits = plan_splits(h, T, b);
+    return MOE_OK;
+}
+
+MOE_API int moe_forward(moe_handle h, int T, const void *x, const float *router_w, const int8_t *w_lin,
+                        const void *s_lin, const int8_t *w_v, const void *s_v, const int8_t *w_1, const void *s_1,
+                        void *out, void *stream)
+{
+    if (!h || T < 0 || T > MOE_MAX_TOKENS) return MOE_EINVAL;
+    if (T == 0) return MOE_OK;
+    if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_EINVAL;
+    int rc = check_weights(h, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1);
+    if (rc != MOE_OK) return rc;
+    const size_t xb = static_cast<size_t>(T) * h->d * 2;
+    if (overlaps(x, xb, out, xb)) return MOE_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((rc = begin_call(h, T, s)) != MOE_OK) return rc;
+    return run_layer(h, T, x, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, out, nullptr, nullptr, 0.f, s);
+}
+
+MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const float *router_w, const int8_t *w_lin,
+                             const void *s_lin, const int8_t *w_v, const void *s_v, const int8_t *w_1,
+                             const void *s_1, void *out_host, void *stream)
+{
+    if (!h || T < 0 || T > MOE_MAX_TOKENS) return MOE_EINVAL;
+    if (T == 0) return MOE_OK;
+    if (!x_host || !out_host) return MOE_EINVAL;
+    int rc = check_weights(h, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((rc = begin_call(h, T, s)) != MOE_OK) return rc;
+    const size_t xb = static_cast<size_t>(T) * h->d * 2;
+    char *xs = static_cast<char *>(h->b_stage.ptr);
+    char *os = xs + xb;
+    if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ECUDA;
+    if ((rc = run_layer(h, T, xs, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, os, nullptr, nullptr, 0.f, s)) != MOE_OK)
+        return rc;
+    if (cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+    return MOE_OK;
+}
+
+MOE_API int moe_block_forward(moe_handle h, int T, void *h_io, const void *g_pre, const void *g_post, float eps,
+                              const float *router_w, const int8_t *w_lin, const void *s_lin, const int8_t *w_v,
+                              const void *s_v, const int8_t *w_1, const void *s_1, void *stream)
+{
+    if (!h || T < 0 || T > MOE_MAX_TOKENS) return MOE_EINVAL;
+    if (T == 0) return MOE_OK;
+    if (!h_io || !g_pre || !g_post || !aligned16(h_io) || !aligned16(g_pre) || !aligned16(g_post)) return MOE_EINVAL;
+    if (!(eps >= 0.f)) return MOE_EINVAL;
+    int rc = check_weights(h, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((rc = begin_call(h, T, s)) != MOE_OK) return rc;
+    __nv_bfloat16 *u = static_cast<__nv_bfloat16 *>(h->b_stage.ptr);
+    NormArgs na{T, h->d, static_cast<const __nv_bfloat16 *>(h_io), static_cast<const __nv_bfloat16 *>(g_pre), eps, u};
+    if (timed(h, K_PRENORM, s, [&] { return launch_prenorm(na, s); }) != cudaSuccess) return MOE_ECUDA;
+    return run_layer(h, T, u, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, nullptr, h_io, g_post, eps, s);
+}
+
+MOE_API int moe_get_routing(moe_handle h, int32_t *idx, float *gate, int32_t *offsets, int32_t *perm, void *stream)
+{
+    if (!h || h->last_T < 0) return MOE_EINVAL;
+    const int T = h->last_T;
+    const RouteLayout L = route_layout(T, h->E);
+    const int *rw = static_cast<const int *>(h->b_route.ptr);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    struct {
+        void *dst;
+        const void *src;
+        size_t bytes;
+    } cp[] = {{idx, rw + L.idx, 2 * static_cast<size_t>(T) * 4},
+              {gate, rw + L.gate, 2 * static_cast<size_t>(T) * 4},
+              {offsets, rw + L.offsets, static_cast<size_t>(h->E + 1) * 4},
+              {perm, rw + L.perm, 2 * static_cast<size_t>(T) * 4}};
+    for (auto &c : cp)
+        if (c.dst && cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return MOE_ECUDA;
+    return MOE_OK;
+}
+
+MOE_API int moe_sync_status(moe_handle h, void *stream)
+{
+    if (!h) return MOE_EINVAL;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ECUDA;
+    if (!h->err) return MOE_OK;
+    int e = 0;
+    if (cudaMemcpy(&e, h->err, sizeof e, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ECUDA;
+    if (e == 0) return MOE_OK;
+    cudaMemset(h->err, 0, sizeof e);
+    return e >= kErrTimeoutBase ? MOE_ETIMEOUT : MOE_ECUDA;
+}
+
+MOE_API int moe_set_profiling(moe_handle h, int on)
+{
+    if (!h) return MOE_EINVAL;
+    h->prof = on != 0;
+    return MOE_OK;
+}
+
+MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n)
+{
+    if (!h || n < 0) return MOE_EINVAL;
+    for (int i = 0; i < n; ++i) {
+        if (ms) ms[i] = 0.f;
+        if (launches) launches[i] = 0;
+    }
+    int rc = MOE_OK;
+    for (auto &p : h->pending) {
+        float t = 0.f;
+        if (cudaEventSynchronize(p.b) != cudaSuccess || cudaEventElapsedTime(&t, p.a, p.b) != cudaSuccess) {
+            cudaGetLastError();
+            rc = MOE_ECUDA;
+        } else if (p.id < n) {
+            if (ms) ms[p.id] += t;
+            if (launches) launches[p.id] += 1;
+        }
+        h->event_pool.push_back(p.a);
+        h->event_pool.push_back(p.b);
+    }
+    h->pending.clear();
+    return rc;
+}
+
+}  // extern "C"

@@ -8,8 +8,21 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _build_all():
+    """Compile the CUDA library and the oracle's C library if their sources changed."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_moe_build", os.path.join(ROOT, "mixture_experts_softmax_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import oracle
+    oracle.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+    _build_all()
 
 
 def _have_gpu():
