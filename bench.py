@@ -43,6 +43,12 @@ def parse():
     p.add_argument("--workload", default="decode", choices=("decode", "prefill", "skewed", "stacked", "tiny"))
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
+    # smaller variants of a workload for profiler captures (never a bench line)
+    p.add_argument("--tokens", type=int, default=None, help="override T")
+    p.add_argument("--ffn", type=int, default=None, help="override the FFN width")
+    p.add_argument("--skip-extras", action="store_true", help="skip the per-kernel and end-to-end passes")
+    p.add_argument("--layout", choices=("out_in", "in_out"), default="out_in",
+                   help="weight layout: out_in = K-major, packed once at load (TMEM path); in_out = as drawn")
     return p.parse_args()
 
 
@@ -212,6 +218,9 @@ def run_native(args, world, rank, local):
     import mixture_experts_softmax_b200 as moe
 
     w = moe_synth.WORKLOADS[args.workload]
+    if args.tokens or args.ffn:
+        import dataclasses
+        w = dataclasses.replace(w, T=args.tokens or w.T, F=args.ffn or w.F, name=w.name + "_resized")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     K, W = args.steps, args.warmup
@@ -226,6 +235,17 @@ def run_native(args, world, rank, local):
 
     h = moe.MoELayer(w.d, w.F, w.E, w.k)
     moe.check(moe.moe_set_router_bias(h.h, bias))
+    if args.layout == "out_in":
+        # one-time weight-load step, outside every timed region: K-major int8 copies
+        moe.check(moe.moe_set_weight_layout(h.h, moe.MOE_LAYOUT_OUT_IN))
+        drawn = layers
+        layers = [moe.pack_layer(h.h, l) for l in drawn]
+        torch.cuda.synchronize(dev)
+        for l in drawn:
+            for k in ("wl", "wv", "w1"):
+                l[k] = None
+        del drawn
+        torch.cuda.empty_cache()
     out = torch.empty_like(inp.x)
     res0 = inp.x.clone()
 
@@ -266,6 +286,12 @@ def run_native(args, world, rank, local):
     ms_max = max_over_ranks(ms, world, dev)
     tokens = T * world
     value = tokens / (ms_max / 1e3)
+
+    if args.skip_extras:
+        h.close()
+        return {"metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": ms_max, "n_gpus": world,
+                "steps": K, "warmup": W, "config": {"workload": w.name, "T_per_gpu": T, "ffn": w.F},
+                "note": "profiling variant: no per-kernel or end-to-end pass"}
 
     # per-kernel durations: the same K steps again with events around every launch
     moe.check(moe.moe_set_profiling(h.h, True))
@@ -344,7 +370,9 @@ def run_native(args, world, rank, local):
         "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded; random-init int8 weights of the Grok-1 MoE shape)",
         "config": {"workload": args.workload, "T_per_gpu": T, "d_model": w.d, "ffn": w.F, "experts": w.E,
-                   "top_k": w.k, "blocks": w.blocks or 1, "weights": "int8 + bf16 per-output-channel scales",
+                   "top_k": w.k, "blocks": w.blocks or 1,
+                   "weights": "int8 + bf16 per-output-channel scales, layout " + args.layout +
+                              (" (packed once at load, untimed)" if args.layout == "out_in" else ""),
                    "l2": "inputs larger than L2 (%.2f GB of weights per step)" % (layer_bytes / 1e9),
                    "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],
                    "down_splits": moe.moe_plan(h.h, T)[2]},

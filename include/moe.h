@@ -63,6 +63,10 @@ extern "C" {
 /* Largest token count one call accepts. */
 #define MOE_MAX_TOKENS   262144
 
+/* Weight layouts (moe_set_weight_layout). */
+#define MOE_LAYOUT_IN_OUT 0   /* w_lin, w_v [E, d, F]; w_1 [E, F, d]  (x @ W orientation, default) */
+#define MOE_LAYOUT_OUT_IN 1   /* w_lin, w_v [E, F, d]; w_1 [E, d, F]  (reduction dim contiguous)  */
+
 typedef struct moe_ctx *moe_handle;
 
 /* Human-readable text for a status code.  Never NULL; the string is static. */
@@ -177,6 +181,29 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns);
  */
 MOE_API int moe_set_profiling(moe_handle h, int on);
 MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
+
+/*
+ * Select how the forward calls of this handle read w_lin, w_v and w_1:
+ *   MOE_LAYOUT_IN_OUT (default)  [E, in, out]: the layout block above;
+ *   MOE_LAYOUT_OUT_IN            [E, out, in]: each output feature's reduction
+ *                                elements contiguous (w_lin, w_v [E, F, d];
+ *                                w_1 [E, d, F]); produced by moe_pack_weight.
+ * Both layouts give the same result up to fp32 summation order.  With
+ * MOE_LAYOUT_OUT_IN the GEMMs keep the dequantised bf16 weights in tensor memory
+ * instead of shared memory, the faster path; the layout change is a one-time
+ * cost at weight-load time.  Scales are the same in both layouts.
+ * Returns MOE_EINVAL for an unknown layout.
+ */
+MOE_API int moe_set_weight_layout(moe_handle h, int layout);
+
+/*
+ * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT to MOE_LAYOUT_OUT_IN
+ * (a per-expert transpose; the values are copied unchanged), enqueued on `stream`.
+ *   which = 0: w is linear or linear_v, [E, d, F] -> w_packed [E, F, d]
+ *   which = 1: w is linear_1,           [E, F, d] -> w_packed [E, d, F]
+ * w and w_packed are device buffers of E*d*F bytes that must not overlap.
+ */
+MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream);
 
 /*
  * The tile shape and split chosen for T tokens (for tests and benchmarks):

@@ -27,6 +27,8 @@ MOE_ECUDA = -4
 MOE_ETIMEOUT = -5
 MOE_ENODEV = -6
 MOE_MAX_TOKENS = 262144
+MOE_LAYOUT_IN_OUT = 0
+MOE_LAYOUT_OUT_IN = 1
 
 KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm")
 
@@ -35,6 +37,7 @@ EXPORTS = (
     "moe_strerror", "moe_version", "moe_create", "moe_destroy", "moe_set_router_bias",
     "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing",
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
+    "moe_set_weight_layout", "moe_pack_weight",
 )
 
 
@@ -47,7 +50,7 @@ class MoEError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m mixture_experts_softmax_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python mixture_experts_softmax_b200/build.py` "
             "(there is no fallback implementation)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
@@ -66,6 +69,8 @@ def _load() -> ctypes.CDLL:
         "moe_set_profiling": (I, [P, I]),
         "moe_get_kernel_times": (I, [P, P, P, I]),
         "moe_plan": (I, [P, I, ctypes.POINTER(I), ctypes.POINTER(I)]),
+        "moe_set_weight_layout": (I, [P, I]),
+        "moe_pack_weight": (I, [P, P, P, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -168,6 +173,28 @@ def moe_get_kernel_times(h):
     cnt = (ctypes.c_int * n)()
     rc = _lib.moe_get_kernel_times(h, ms, cnt, n)
     return rc, {KERNEL_NAMES[i]: (ms[i], cnt[i]) for i in range(n)}
+
+
+def moe_set_weight_layout(h, layout: int) -> int:
+    return _lib.moe_set_weight_layout(h, int(layout))
+
+
+def moe_pack_weight(h, w, w_packed, which: int, stream=None) -> int:
+    return _lib.moe_pack_weight(h, _ptr(w), _ptr(w_packed), int(which), _stream(stream))
+
+
+def pack_layer(h, layer: dict, stream=None) -> dict:
+    """A copy of `layer` with its three int8 weights rewritten to MOE_LAYOUT_OUT_IN
+    (new device buffers; scales and router weight shared with `layer`)."""
+    import torch
+    out = dict(layer)
+    for key, which in (("wl", 0), ("wv", 0), ("w1", 1)):
+        w = layer[key]
+        E, a, b = w.shape
+        p = torch.empty((E, b, a), dtype=torch.int8, device=w.device)
+        check(moe_pack_weight(h, w, p, which, stream), "moe_pack_weight")
+        out[key] = p
+    return out
 
 
 def moe_plan(h, T: int):

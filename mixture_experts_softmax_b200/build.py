@@ -1,6 +1,6 @@
 """Compile the CUDA library in place with nvcc for sm_100a.
 
-    python -m mixture_experts_softmax_b200.build
+    python mixture_experts_softmax_b200/build.py
 
 Produces ``libmoe_b200.so`` next to this file.  The CUDA runtime is linked
 statically, so loading the library needs no GPU and no libcudart on the path.

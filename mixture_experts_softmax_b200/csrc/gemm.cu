@@ -14,7 +14,7 @@
 // Per pipeline stage (kBK = 64 reduction elements):
 //   - a TMA producer thread copies the int8 weight tile(s) [64 k x 128 f] into a
 //     staging ring (128-byte swizzle);
-//   - 8 converter warps turn each int8 tile into bf16 in the canonical
+//   - 16 converter warps turn each int8 tile into bf16 in the canonical
 //     MN-major 128-byte-swizzled UMMA layout (int8 -> bf16 is exact);
 //   - a second TMA producer thread copies the bf16 activation tile [BN r x 64 k]
 //     (K-major, 128-byte swizzle) straight into the operand ring;
@@ -29,27 +29,19 @@
 // on the device from the padded expert offsets.  Every wait on an mbarrier is
 // bounded in time; on expiry the kernel records an error, stops, drains its own
 // in-flight copies and MMAs and frees TMEM.
-#include "kernels.cuh"
-#include "ptx.cuh"
+#include "gemm_common.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kThreads = 512;                  // 16 warps
+constexpr int kThreads = 768;                  // 24 warps
 constexpr int kWarpTmaA = 0, kWarpMma = 1, kWarpTmaB = 2;
 constexpr int kWarpEpi0 = 4;                   // warps 4..7: epilogue (TMEM lanes 0..127)
-constexpr int kWarpConv0 = 8;                  // warps 8..15: int8 -> bf16 converters
+constexpr int kWarpConv0 = 8;                  // warps 8..23: int8 -> bf16 converters
 constexpr int kConvThreads = (kThreads / 32 - kWarpConv0) * 32;
+static_assert(kConvThreads == kBM * kBK / 16, "one 16-byte unit per converter thread and matrix");
 constexpr int kSmemBudget = 216 * 1024;
-
-constexpr int cmin(int a, int b) { return a < b ? a : b; }
-constexpr int pow2_at_least(int v)
-{
-    int p = 32;
-    while (p < v) p <<= 1;
-    return p;
-}
 
 template <bool UP, int BN>
 struct Cfg {
@@ -76,86 +68,12 @@ struct Cfg {
     static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
 };
 
-// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version bits.
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo)
-{
-    return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(lbo >> 4) << 16) |
-           (static_cast<uint64_t>(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
-
 // kind::f16 instruction descriptor: D fp32, A and B bf16, A MN-major, B K-major, M = 128.
 template <int BN>
 __device__ __forceinline__ constexpr uint32_t idesc_bf16()
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (static_cast<uint32_t>(BN >> 3) << 17) |
            (static_cast<uint32_t>(kBM >> 4) << 24);
-}
-
-// Two signed bytes (chosen by `sel`) -> two exact bf16 values.  With the byte b in
-// the low 7 mantissa bits under exponent 2^7, hi = 128 + (b & 127); lo is 128, or
-// 256 when b's sign bit is set (it lands on the exponent's lowest bit); hi - lo = b
-// exactly (an integer of at most 8 significant bits).
-__device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w, uint32_t sel)
-{
-    const uint32_t p = __byte_perm(w, 0x43434343u, sel);
-    const uint32_t hi = p & 0xFF7FFF7Fu;
-    const uint32_t lo = p & 0xFF80FF80u;
-    __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&hi),
-                               *reinterpret_cast<const __nv_bfloat162 *>(&lo));
-    return *reinterpret_cast<uint32_t *>(&r);
-}
-
-__device__ __forceinline__ float gelu_tanh(float a)
-{
-    // 0.5 a (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3)))
-    const float k0 = 0.7978845608028654f, k1 = 0.044715f * 0.7978845608028654f;
-    const float u = a * fmaf(k1, a * a, k0);
-    const float h = 0.5f * a;
-    return fmaf(h, tanh_approx(u), h);
-}
-
-struct Waiter {
-    volatile uint32_t *abort;
-    int *err;
-    long long timeout_ns;
-
-    // wait for the phase of `bar` with parity `par`; false if the CTA aborted or the limit ran out
-    __device__ __forceinline__ bool wait(uint32_t bar, uint32_t par, int site) const
-    {
-        if (mbar_try_wait(bar, par)) return true;
-        const uint64_t t0 = global_timer_ns();
-        while (true) {
-            if (mbar_try_wait(bar, par)) return true;
-            if (*abort) return false;
-            if (static_cast<long long>(global_timer_ns() - t0) > timeout_ns) {
-                *abort = 1u;
-                atomicCAS(err, 0, kErrTimeoutBase + site);
-                return false;
-            }
-        }
-    }
-};
-
-// wait used only while draining after an abort: fixed 1 s limit, ignores the abort flag
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t par)
-{
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, par))
-        if (global_timer_ns() - t0 > 1000000000ull) return;
-}
-
-template <int BN>
-__device__ __forceinline__ void decode_tile(int tile, const int *prefix, const int *poff, int m_tiles,
-                                            int splits, int &e, int &m, int &n, int &s)
-{
-    e = 0;
-    while (tile >= prefix[e + 1]) ++e;
-    int local = tile - prefix[e];
-    s = local % splits;
-    local /= splits;
-    const int nt = (poff[e + 1] - poff[e]) / BN;
-    n = local % nt;
-    m = local / nt;
 }
 
 template <bool UP, int BN>
@@ -221,7 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     const int total = prefix[a.E];
-    const Waiter w{abort_flag, a.err, a.timeout_ns};
+#ifdef MOE_PIPE_STATS
+    if (threadIdx.x == 0) atomicAdd(&g_pipe_stats[UP ? 28 : 29], static_cast<unsigned long long>(clock64()));
+#endif
+    const Waiter w{abort_flag, a.err, a.timeout_ns, UP ? 0 : 10};
 
     if (warp == kWarpTmaA) {
         // ---- int8 weight tiles -> staging ring ------------------------------------
@@ -367,40 +288,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= kWarpConv0) {
         // ---- int8 staging -> bf16 UMMA operand (MN-major, 128-byte swizzle) --------
-        // unit u of 512 per matrix: reduction row k = (u & 7) | (u >> 6) << 3 and a
-        // 16-feature chunk mc = (u >> 3) & 7; 8 consecutive lanes take 8 rows of one
-        // chunk, so both the swizzled reads and the swizzled writes are conflict-free.
+        // Thread ct owns one 16-byte unit of every [64 k x 128 f] int8 tile: reduction
+        // row k = (ct & 7) | (ct >> 6) << 3 and 16-feature chunk mc = (ct >> 3) & 7.
+        // 8 consecutive lanes take 8 rows of one chunk, so both the swizzled reads and
+        // the swizzled writes are free of bank conflicts.
         const int ct = threadIdx.x - kWarpConv0 * 32;
+        const int k = (ct & 7) | ((ct >> 6) << 3);
+        const int mc = (ct >> 3) & 7;
+        const int kr = k & 7;
+        const uint32_t src_off = k * 128 + ((mc ^ kr) << 4);
+        const uint32_t atom = ((((k >> 3) * 2 + (mc >> 2)) << 10) + kr * 128);
+        const uint32_t dst_lo = atom + ((((mc & 3) * 2) ^ kr) << 4);
+        const uint32_t dst_hi = atom + (((((mc & 3) * 2) ^ kr) ^ 1) << 4);
         uint32_t st = 0, ph = 0, st2 = 0, ph2 = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             bool ok = true;
             for (int ks = 0; ks < a.ksteps; ++ks) {
                 ok = __all_sync(0xffffffffu, w.wait(stg_full(st), ph, 7) && w.wait(op_empty(st2), ph2 ^ 1u, 8));
                 if (!ok) break;
-                const uint32_t src0 = sbase + C::OFF_STG + st * C::STG;
+                const uint32_t src0 = sbase + C::OFF_STG + st * C::STG + src_off;
                 const uint32_t dst0 = sbase + C::OFF_A + st2 * C::ABYTES;
+                uint4 v[C::NA];
+#pragma unroll
+                for (int mat = 0; mat < C::NA; ++mat) v[mat] = lds128(src0 + mat * kBM * kBK);
 #pragma unroll
                 for (int mat = 0; mat < C::NA; ++mat) {
-#pragma unroll
-                    for (int u = ct; u < 512; u += kConvThreads) {
-                        const int k = (u & 7) | ((u >> 6) << 3);
-                        const int mc = (u >> 3) & 7;
-                        const int kr = k & 7;
-                        const uint4 v = lds128(src0 + mat * kBM * kBK + k * 128 + ((mc ^ kr) << 4));
-                        uint4 lo, hi;
-                        lo.x = i8x2_to_bf16x2(v.x, 0x4140);
-                        lo.y = i8x2_to_bf16x2(v.x, 0x4342);
-                        lo.z = i8x2_to_bf16x2(v.y, 0x4140);
-                        lo.w = i8x2_to_bf16x2(v.y, 0x4342);
-                        hi.x = i8x2_to_bf16x2(v.z, 0x4140);
-                        hi.y = i8x2_to_bf16x2(v.z, 0x4342);
-                        hi.z = i8x2_to_bf16x2(v.w, 0x4140);
-                        hi.w = i8x2_to_bf16x2(v.w, 0x4342);
-                        const uint32_t atom = dst0 + mat * kBM * kBK * 2 + (((k >> 3) * 2 + (mc >> 2)) << 10) + kr * 128;
-                        const int c0 = ((mc & 3) * 2) ^ kr;
-                        sts128(atom + (c0 << 4), lo);
-                        sts128(atom + ((c0 ^ 1) << 4), hi);
-                    }
+                    uint4 lo, hi;
+                    lo.x = i8x2_to_bf16x2(v[mat].x, 0x4140);
+                    lo.y = i8x2_to_bf16x2(v[mat].x, 0x4342);
+                    lo.z = i8x2_to_bf16x2(v[mat].y, 0x4140);
+                    lo.w = i8x2_to_bf16x2(v[mat].y, 0x4342);
+                    hi.x = i8x2_to_bf16x2(v[mat].z, 0x4140);
+                    hi.y = i8x2_to_bf16x2(v[mat].z, 0x4342);
+                    hi.z = i8x2_to_bf16x2(v[mat].w, 0x4140);
+                    hi.w = i8x2_to_bf16x2(v[mat].w, 0x4342);
+                    const uint32_t d = dst0 + mat * kBM * kBK * 2;
+                    sts128(d + dst_lo, lo);
+                    sts128(d + dst_hi, hi);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -421,6 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
+#ifdef MOE_PIPE_STATS
+    if (threadIdx.x == 0) atomicAdd(&g_pipe_stats[UP ? 30 : 31], static_cast<unsigned long long>(clock64()));
+#endif
 }
 
 template <bool UP, int BN>
@@ -476,3 +403,18 @@ cudaError_t launch_gemm_down(int bn, const CUtensorMap &w1, const CUtensorMap &h
 }
 
 }  // namespace moe
+
+#ifdef MOE_PIPE_STATS
+// instrumented builds only: copy (and optionally clear) the per-site wait-cycle sums
+extern "C" __attribute__((visibility("default"))) int moe_debug_pipe_stats(unsigned long long *out, int reset)
+{
+    if (cudaMemcpyFromSymbol(out, moe::g_pipe_stats, sizeof(unsigned long long) * 64) != cudaSuccess) return -4;
+    if (reset) {
+        unsigned long long z[64] = {};
+        if (cudaMemcpyToSymbol(moe::g_pipe_stats, z, sizeof z) != cudaSuccess) return -4;
+    }
+    return 0;
+}
+#endif
+
+

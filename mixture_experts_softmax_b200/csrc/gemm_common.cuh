@@ -1,0 +1,112 @@
+// gemm_common.cuh -- pieces shared by the two grouped-GEMM kernels (weights from the
+// reference [E, in, out] layout through shared memory, and pre-packed K-major weights
+// through TMEM): descriptors, the int8 -> bf16 conversion, GELU, bounded waits and the
+// device-side tile list.
+#pragma once
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+constexpr int pow2_at_least(int v)
+{
+    int p = 32;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+#ifdef MOE_PIPE_STATS
+// cycles spent in each wait site, summed over the CTA (instrumented builds only; one
+// array per translation unit)
+static __device__ unsigned long long g_pipe_stats[64];
+#endif
+
+// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version bits.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(lbo >> 4) << 16) |
+           (static_cast<uint64_t>(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Two signed bytes (chosen by `sel`) -> two exact bf16 values.  With the byte b in
+// the low 7 mantissa bits under exponent 2^7, hi = 128 + (b & 127); lo is 128, or
+// 256 when b's sign bit is set (it lands on the exponent's lowest bit); hi - lo = b
+// exactly (an integer of at most 8 significant bits).
+__device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w, uint32_t sel)
+{
+    const uint32_t p = __byte_perm(w, 0x43434343u, sel);
+    const uint32_t hi = p & 0xFF7FFF7Fu;
+    const uint32_t lo = p & 0xFF80FF80u;
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&hi),
+                               *reinterpret_cast<const __nv_bfloat162 *>(&lo));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ float gelu_tanh(float a)
+{
+    // 0.5 a (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3)))
+    const float k0 = 0.7978845608028654f, k1 = 0.044715f * 0.7978845608028654f;
+    const float u = a * fmaf(k1, a * a, k0);
+    const float h = 0.5f * a;
+    return fmaf(h, tanh_approx(u), h);
+}
+
+struct Waiter {
+    volatile uint32_t *abort;
+    int *err;
+    long long timeout_ns;
+    int stat_base;   // instrumented builds: first stats slot of this kernel
+
+    // wait for the phase of `bar` with parity `par`; false if the CTA aborted or the limit ran out
+    __device__ __forceinline__ bool wait(uint32_t bar, uint32_t par, int site) const
+    {
+        if (mbar_try_wait(bar, par)) return true;
+#ifdef MOE_PIPE_STATS
+        const long long c0 = clock64();
+        const bool ok = wait_slow(bar, par, site);
+        atomicAdd(&g_pipe_stats[stat_base + site], static_cast<unsigned long long>(clock64() - c0));
+        return ok;
+    }
+
+    __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t par, int site) const
+    {
+#endif
+        const uint64_t t0 = global_timer_ns();
+        while (true) {
+            if (mbar_try_wait(bar, par)) return true;
+            if (*abort) return false;
+            if (static_cast<long long>(global_timer_ns() - t0) > timeout_ns) {
+                *abort = 1u;
+                atomicCAS(err, 0, kErrTimeoutBase + site);
+                return false;
+            }
+        }
+    }
+};
+
+// wait used only while draining after an abort: fixed 1 s limit, ignores the abort flag
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t par)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, par))
+        if (global_timer_ns() - t0 > 1000000000ull) return;
+}
+
+template <int BN>
+__device__ __forceinline__ void decode_tile(int tile, const int *prefix, const int *poff, int m_tiles,
+                                            int splits, int &e, int &m, int &n, int &s)
+{
+    e = 0;
+    while (tile >= prefix[e + 1]) ++e;
+    int local = tile - prefix[e];
+    s = local % splits;
+    local /= splits;
+    const int nt = (poff[e + 1] - poff[e]) / BN;
+    n = local % nt;
+    m = local / nt;
+}
+
+
+}  // namespace moe

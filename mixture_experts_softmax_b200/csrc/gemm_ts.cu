@@ -1,0 +1,413 @@
+// gemm_ts.cu -- grouped expert GEMMs for int8 weights stored K-major ([E, out, in], one
+// row of reduction elements per output feature), with the dequantised bf16 weights
+// kept in tensor memory (TMEM) as the MMA's A operand.
+//
+// Computes the expert MLP of "Grok-1 Admin & Architecture Guide", section 3,
+// "Mixture of Experts (MoELayer + Router)" step 3, linear_1(gelu(linear(x)) * linear_v(x)),
+// with the 8-bit weights of section 3 "Quantized weights" (int8 value * scale).
+//
+// Same tile orientation as the shared-memory variant (weights = A, M = 128 output
+// features; grouped token rows = B, N = BN rows), but per pipeline stage of 128
+// reduction elements:
+//   - a TMA producer thread copies the int8 weight tile(s) [128 f x 128 k] (128-byte
+//     swizzle) into a shared-memory staging ring;
+//   - 16 converter warps each own 32 feature rows (one TMEM lane quadrant) and a slice
+//     of the 128 reduction elements: they read their bytes from the staging tile,
+//     convert int8 -> bf16 exactly and store the bf16 pairs into the A ring in TMEM
+//     with tcgen05.st (one 32-bit TMEM column holds two consecutive k);
+//   - a second TMA producer copies the bf16 activation tile [BN r x 128 k] into the
+//     shared-memory operand ring;
+//   - one thread issues tcgen05.mma with A from TMEM and B from shared memory;
+//   - 4 epilogue warps apply the same fused epilogues as the shared-memory variant.
+// Shared-memory traffic per weight byte is the TMA write plus one read (against
+// also a bf16 write and an MMA read of 2 bytes each when the dequantised tile goes
+// through shared memory), which takes shared-memory bandwidth off the critical path.
+#include "gemm_common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 768;                  // 24 warps
+constexpr int kWarpTmaA = 0, kWarpMma = 1, kWarpTmaB = 2;
+constexpr int kWarpEpi0 = 4;                   // warps 4..7: epilogue (TMEM lanes 0..127)
+constexpr int kWarpConv0 = 8;                  // warps 8..23: converters
+constexpr int kConvWarps = 16;
+constexpr int kBKT = 128;                      // reduction elements per stage
+constexpr int kSmemBudget = 208 * 1024;
+static_assert(kWarpConv0 % 4 == 0, "converter warp w must own TMEM lane quadrant w % 4");
+
+template <bool UP, int BN>
+struct CfgTS {
+    static constexpr int NA = UP ? 2 : 1;                   // weight matrices per stage
+    static constexpr int KP = kConvWarps / 4 / NA;          // converter warps per (quadrant, matrix)
+    static constexpr int CH = (kBKT / 16) / KP;             // 16-byte chunks per converter thread and stage
+    static constexpr int STG = NA * kBM * kBKT;             // int8 staging bytes per stage
+    static constexpr int BBYTES = BN * kBKT * 2;            // bf16 activation bytes per stage
+    static constexpr int NDB = (UP && BN == 128) ? 1 : 2;   // accumulator buffers in TMEM
+    static constexpr int ACC = NA * BN;                     // TMEM columns of one accumulator buffer
+    static constexpr int A_COLS = NA * kBKT / 2;            // TMEM columns of one A stage
+    static constexpr int S2 = cmin(4, (512 - NDB * ACC) / A_COLS);   // A (TMEM) + B (smem) ring
+    static constexpr int S1 = cmin(12, (kSmemBudget - S2 * BBYTES) / STG);   // int8 staging ring
+    static constexpr int A_BASE = NDB * ACC;                // first TMEM column of the A ring
+    static constexpr int TMEM_COLS = pow2_at_least(NDB * ACC + S2 * A_COLS);
+    static constexpr int OFF_STG = 0;
+    static constexpr int OFF_B = OFF_STG + S1 * STG;
+    static constexpr int OFF_BAR = OFF_B + S2 * BBYTES;
+    // barriers: stg_full[S1] stg_empty[S1] a_full[S2] b_full[S2] op_empty[S2] acc_full[NDB] acc_empty[NDB] drain
+    static constexpr int NBAR = 2 * S1 + 3 * S2 + 2 * NDB + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int MISC_BYTES = 16 + 2 * 4 * 40;
+    static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;
+    static_assert(S1 >= 2 && S2 >= 2, "rings too shallow");
+    static_assert(SMEM <= 227 * 1024, "shared memory over the per-CTA limit");
+    static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
+    static_assert(CH * 8 == 16 || CH * 8 == 32, "a converter thread stores 16 or 32 TMEM columns");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is 16..256 in steps of 16");
+};
+
+// kind::f16 instruction descriptor: D fp32, A and B bf16, both K-major, M = 128.
+template <int BN>
+__device__ __forceinline__ constexpr uint32_t idesc_ts()
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+           (static_cast<uint32_t>(kBM >> 4) << 24);
+}
+
+template <bool UP, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_ts_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, const GemmArgs a)
+{
+    using C = CfgTS<UP, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
+    auto stg_full = [&](int s) { return bar(s); };
+    auto stg_empty = [&](int s) { return bar(C::S1 + s); };
+    auto a_full = [&](int s) { return bar(2 * C::S1 + s); };
+    auto b_full = [&](int s) { return bar(2 * C::S1 + C::S2 + s); };
+    auto op_empty = [&](int s) { return bar(2 * C::S1 + 2 * C::S2 + s); };
+    auto acc_full = [&](int b) { return bar(2 * C::S1 + 3 * C::S2 + b); };
+    auto acc_empty = [&](int b) { return bar(2 * C::S1 + 3 * C::S2 + C::NDB + b); };
+    const uint32_t drain_bar = bar(2 * C::S1 + 3 * C::S2 + 2 * C::NDB);
+
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile uint32_t *abort_flag = misc + 1;
+    int *prefix = reinterpret_cast<int *>(misc + 4);
+    int *poff = prefix + 40;
+    const int m_tiles = a.M / kBM;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::S1; ++s) {
+            mbar_init(stg_full(s), 1);
+            mbar_init(stg_empty(s), kConvWarps);
+        }
+        for (int s = 0; s < C::S2; ++s) {
+            mbar_init(a_full(s), kConvWarps);
+            mbar_init(b_full(s), 1);
+            mbar_init(op_empty(s), 1);
+        }
+        for (int b = 0; b < C::NDB; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), 4);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0u;
+        prefix[0] = 0;
+        for (int e = 0; e <= a.E; ++e) poff[e] = a.poff[e];
+        for (int e = 0; e < a.E; ++e)
+            prefix[e + 1] = prefix[e] + m_tiles * ((poff[e + 1] - poff[e]) / BN) * a.splits;
+        fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32(misc), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == kWarpTmaA && lane == 0) {
+        prefetch_tmap(&tmA0);
+        if (UP) prefetch_tmap(&tmA1);
+        prefetch_tmap(&tmB);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = misc[0];
+    const int total = prefix[a.E];
+#ifdef MOE_PIPE_STATS
+    if (threadIdx.x == 0) atomicAdd(&g_pipe_stats[UP ? 60 : 61], static_cast<unsigned long long>(clock64()));
+#endif
+    const Waiter w{abort_flag, a.err, a.timeout_ns, UP ? 20 : 40};
+
+    if (warp == kWarpTmaA) {
+        // ---- int8 weight tiles [128 f x 128 k] -> staging ring ------------------------
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            uint32_t st = 0, ph = 0, issued = 0, par = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+                int e, m, n, s;
+                decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                const int kb = s * a.ksteps;
+                const int y = e * a.M + m * kBM;
+                for (int ks = 0; ks < a.ksteps; ++ks) {
+                    if (!w.wait(stg_empty(st), ph ^ 1u, 1)) goto a_done;
+                    mbar_arrive_expect_tx(stg_full(st), C::STG);
+                    const uint32_t dst = sbase + C::OFF_STG + st * C::STG;
+                    tma_load_2d(dst, &tmA0, stg_full(st), (kb + ks) * kBKT, y, pol);
+                    if (UP) tma_load_2d(dst + kBM * kBKT, &tmA1, stg_full(st), (kb + ks) * kBKT, y, pol);
+                    issued |= 1u << st;
+                    par = (par & ~(1u << st)) | (ph << st);
+                    if (++st == C::S1) { st = 0; ph ^= 1u; }
+                }
+            }
+        a_done:
+            for (int s = 0; s < C::S1; ++s)   // every copy issued has landed before the CTA may exit
+                if (issued & (1u << s)) wait_drain(stg_full(s), (par >> s) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == kWarpTmaB) {
+        // ---- bf16 activation tiles [BN r x 128 k] (two 64-wide boxes) -> operand ring --
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_last();
+            uint32_t st = 0, ph = 0, issued = 0, par = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+                int e, m, n, s;
+                decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                const int kb = s * a.ksteps;
+                const int row = poff[e] + n * BN;
+                for (int ks = 0; ks < a.ksteps; ++ks) {
+                    if (!w.wait(op_empty(st), ph ^ 1u, 2)) goto b_done;
+                    mbar_arrive_expect_tx(b_full(st), C::BBYTES);
+                    const uint32_t dst = sbase + C::OFF_B + st * C::BBYTES;
+                    const int x = (kb + ks) * kBKT;
+                    tma_load_2d(dst, &tmB, b_full(st), x, row, pol);
+                    tma_load_2d(dst + BN * 128, &tmB, b_full(st), x + 64, row, pol);
+                    issued |= 1u << st;
+                    par = (par & ~(1u << st)) | (ph << st);
+                    if (++st == C::S2) { st = 0; ph ^= 1u; }
+                }
+            }
+        b_done:
+            for (int s = 0; s < C::S2; ++s)
+                if (issued & (1u << s)) wait_drain(b_full(s), (par >> s) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == kWarpMma) {
+        // ---- tensor-core issue: A from TMEM, B from shared memory --------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_ts<BN>();
+            uint32_t st = 0, ph = 0;
+            int it = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+                const int b = it % C::NDB;
+                const uint32_t aph = (it / C::NDB) & 1;
+                if (!w.wait(acc_empty(b), aph ^ 1u, 3)) break;
+                tc_fence_after();
+                const uint32_t dcol = tmem_base + b * C::ACC;
+                bool ok = true;
+                for (int ks = 0; ks < a.ksteps; ++ks) {
+                    if (!w.wait(a_full(st), ph, 4) || !w.wait(b_full(st), ph, 5)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t acol = tmem_base + C::A_BASE + st * C::A_COLS;
+                    const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
+#pragma unroll
+                    for (int kk = 0; kk < kBKT / 16; ++kk) {
+                        const uint64_t bdesc = desc_sw128(bbase + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
+#pragma unroll
+                        for (int mat = 0; mat < C::NA; ++mat)
+                            umma_bf16_ts(dcol + mat * BN, acol + mat * (kBKT / 2) + kk * 8, bdesc, idesc,
+                                         (ks | kk) != 0);
+                    }
+                    umma_commit(op_empty(st));
+                    if (++st == C::S2) { st = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit(acc_full(b));
+            }
+            umma_commit(drain_bar);          // all MMAs issued above have completed after this
+            wait_drain(drain_bar, 0);
+        }
+        __syncwarp();
+    } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
+        // ---- epilogue: TMEM -> registers -> global -----------------------------------
+        const int ew = warp - kWarpEpi0;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+            int e, m, n, s;
+            decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+            const int b = it % C::NDB;
+            const uint32_t aph = (it / C::NDB) & 1;
+            const bool ok = __all_sync(0xffffffffu, w.wait(acc_full(b), aph, 6));
+            if (!ok) break;
+            tc_fence_after();
+            const int f = m * kBM + ew * 32 + lane;
+            const uint32_t tl = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * C::ACC;
+            const int row0 = poff[e] + n * BN;
+            if constexpr (UP) {
+                const float sa = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
+                const float sb = __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float va[16], vb[16];
+                    tmem_ld16(tl + c, va);
+                    tmem_ld16(tl + BN + c, vb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int r = row0 + c + i;
+                        if (__ldg(a.rperm + r) >= 0)
+                            a.h[static_cast<size_t>(r) * a.M + f] =
+                                __float2bfloat16_rn(gelu_tanh(sa * va[i]) * (sb * vb[i]));
+                    }
+                }
+            } else {
+                const float sc = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    tmem_ld16(tl + c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int route = __ldg(a.rperm + row0 + c + i);
+                        if (route >= 0) {
+                            const float g = __ldg(a.gate + route);
+                            const size_t o = ((static_cast<size_t>(s) * a.T + (route >> 1)) * 2 + (route & 1)) *
+                                                 static_cast<size_t>(a.M) + f;
+                            a.slots[o] = g * (sc * v[i]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(b));
+        }
+    } else if (warp >= kWarpConv0) {
+        // ---- int8 staging -> bf16 A operand in TMEM ------------------------------------
+        // Converter warp cw owns TMEM lane quadrant q = warp % 4 (feature rows 32q..32q+31
+        // of the tile), weight matrix `mat` and chunks [j0, j0 + CH) of the 8 16-byte
+        // chunks of each 128-byte feature row.  Lanes of one 8-lane phase read 8
+        // different rows, whose 128-byte swizzle puts the same logical chunk in 8
+        // different bank groups.
+        const int cw = warp - kWarpConv0;
+        const int q = warp & 3;
+        const int part = cw >> 2;
+        const int mat = part / C::KP;
+        const int j0 = (part % C::KP) * C::CH;
+        const int fr = q * 32 + lane;
+        const uint32_t src_row = mat * kBM * kBKT + fr * 128;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        uint32_t st = 0, ph = 0, st2 = 0, ph2 = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            bool ok = true;
+            for (int ks = 0; ks < a.ksteps; ++ks) {
+                ok = __all_sync(0xffffffffu, w.wait(stg_full(st), ph, 7) && w.wait(op_empty(st2), ph2 ^ 1u, 8));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t src = sbase + C::OFF_STG + st * C::STG + src_row;
+                uint4 v[C::CH];
+#pragma unroll
+                for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
+                uint32_t words[C::CH * 8];
+#pragma unroll
+                for (int c = 0; c < C::CH; ++c) {
+                    words[c * 8 + 0] = i8x2_to_bf16x2(v[c].x, 0x4140);
+                    words[c * 8 + 1] = i8x2_to_bf16x2(v[c].x, 0x4342);
+                    words[c * 8 + 2] = i8x2_to_bf16x2(v[c].y, 0x4140);
+                    words[c * 8 + 3] = i8x2_to_bf16x2(v[c].y, 0x4342);
+                    words[c * 8 + 4] = i8x2_to_bf16x2(v[c].z, 0x4140);
+                    words[c * 8 + 5] = i8x2_to_bf16x2(v[c].z, 0x4342);
+                    words[c * 8 + 6] = i8x2_to_bf16x2(v[c].w, 0x4140);
+                    words[c * 8 + 7] = i8x2_to_bf16x2(v[c].w, 0x4342);
+                }
+                const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + mat * (kBKT / 2) + j0 * 8;
+                if constexpr (C::CH * 8 == 32)
+                    tmem_st32(taddr, words);
+                else
+                    tmem_st16(taddr, words);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(stg_empty(st));
+                    mbar_arrive(a_full(st2));
+                }
+                if (++st == C::S1) { st = 0; ph ^= 1u; }
+                if (++st2 == C::S2) { st2 = 0; ph2 ^= 1u; }
+            }
+            if (!ok) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+#ifdef MOE_PIPE_STATS
+    if (threadIdx.x == 0) atomicAdd(&g_pipe_stats[UP ? 62 : 63], static_cast<unsigned long long>(clock64()));
+#endif
+}
+
+template <bool UP, int BN>
+cudaError_t launch_one_ts(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b, const GemmArgs &args,
+                          int grid, cudaStream_t s)
+{
+    using C = CfgTS<UP, BN>;
+    static bool configured = false;   // the attribute is the same for every launch in the process
+    if (!configured) {
+        cudaError_t e =
+            cudaFuncSetAttribute(gemm_ts_kernel<UP, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    gemm_ts_kernel<UP, BN><<<grid, kThreads, C::SMEM, s>>>(a0, a1, b, args);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int gemm_ts_kstep() { return kBKT; }
+
+cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
+                              const GemmArgs &a, int grid, cudaStream_t s)
+{
+    switch (bn) {
+    case 16: return launch_one_ts<true, 16>(wl, wv, xp, a, grid, s);
+    case 32: return launch_one_ts<true, 32>(wl, wv, xp, a, grid, s);
+    case 64: return launch_one_ts<true, 64>(wl, wv, xp, a, grid, s);
+    case 128: return launch_one_ts<true, 128>(wl, wv, xp, a, grid, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a, int grid,
+                                cudaStream_t s)
+{
+    switch (bn) {
+    case 16: return launch_one_ts<false, 16>(w1, w1, h, a, grid, s);
+    case 32: return launch_one_ts<false, 32>(w1, w1, h, a, grid, s);
+    case 64: return launch_one_ts<false, 64>(w1, w1, h, a, grid, s);
+    case 128: return launch_one_ts<false, 128>(w1, w1, h, a, grid, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moe
+
+#ifdef MOE_PIPE_STATS
+extern "C" __attribute__((visibility("default"))) int moe_debug_pipe_stats_ts(unsigned long long *out, int reset)
+{
+    if (cudaMemcpyFromSymbol(out, moe::g_pipe_stats, sizeof(unsigned long long) * 64) != cudaSuccess) return -4;
+    if (reset) {
+        unsigned long long z[64] = {};
+        if (cudaMemcpyToSymbol(moe::g_pipe_stats, z, sizeof z) != cudaSuccess) return -4;
+    }
+    return 0;
+}
+#endif

@@ -92,6 +92,14 @@ cudaError_t launch_gemm_up(int bn, const CUtensorMap &wl, const CUtensorMap &wv,
                            const GemmArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_gemm_down(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,
                              int grid, cudaStream_t s);
+// the same GEMMs for K-major ([E, out, in]) weights, dequantised into TMEM
+cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
+                              const GemmArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,
+                                int grid, cudaStream_t s);
+int gemm_ts_kstep();   // reduction elements per pipeline stage of the TMEM-operand GEMMs
+// out[e, m, k] = in[e, k, m] for E int8 [K, M] matrices (K, M multiples of 64)
+cudaError_t launch_transpose_i8(const int8_t *in, int8_t *out, int E, int K, int M, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_prenorm(const NormArgs &a, cudaStream_t s);
 

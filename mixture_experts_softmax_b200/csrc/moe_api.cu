@@ -23,7 +23,8 @@ struct DevBuf {
 
 struct WeightMap {
     const void *ptr = nullptr;
-    int kind = -1;   // 0: [E*d, F] (linear, linear_v)   1: [E*F, d] (linear_1)
+    int kind = -1;     // 0: linear / linear_v   1: linear_1
+    int layout = -1;   // MOE_LAYOUT_IN_OUT or MOE_LAYOUT_OUT_IN
     CUtensorMap map;
 };
 
@@ -61,6 +62,7 @@ struct moe_ctx {
 
     const float *bias = nullptr;
     long long timeout_ns = 2000000000LL;
+    int layout = MOE_LAYOUT_IN_OUT;
 
     // profiling
     bool prof = false;
@@ -82,12 +84,14 @@ int plan_bn(int T)
 
 int bn_slot(int bn) { return bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3; }
 
+int kstep_of(const moe_ctx *h) { return h->layout == MOE_LAYOUT_OUT_IN ? gemm_ts_kstep() : kBK; }
+
 int plan_splits(const moe_ctx *h, int T, int bn)
 {
     const int per_expert = (2 * T + h->E - 1) / h->E;
     const long nt = per_expert <= bn ? 1 : (per_expert + bn - 1) / bn;
     const long tiles = static_cast<long>(h->E) * (h->d / kBM) * nt;
-    const int ksteps = h->F / kBK;
+    const int ksteps = h->F / kstep_of(h);
     const int sms = h->num_sms > 0 ? h->num_sms : 148;
     int s = 1;
     while (s < kMaxSplits && tiles * s < 16L * sms && ksteps % (2 * s) == 0) s *= 2;
@@ -227,19 +231,27 @@ int encode_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *ptr
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ECUDA;
 }
 
+// int8 weight descriptor.  [E, in, out] layout: rows = E*in, box = 64 k-rows x 128 features.
+// [E, out, in] layout: rows = E*out, box = 128 feature-rows x 128 k.
 int weight_map(moe_ctx *h, const void *ptr, int kind, const CUtensorMap **out)
 {
     for (auto &w : h->wmaps)
-        if (w.ptr == ptr && w.kind == kind) {
+        if (w.ptr == ptr && w.kind == kind && w.layout == h->layout) {
             *out = &w.map;
             return MOE_OK;
         }
     WeightMap w;
     w.ptr = ptr;
     w.kind = kind;
-    const uint64_t rows = kind == 0 ? static_cast<uint64_t>(h->E) * h->d : static_cast<uint64_t>(h->E) * h->F;
-    const uint64_t cols = kind == 0 ? h->F : h->d;
-    int rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, cols, rows, kBM, kBK);
+    w.layout = h->layout;
+    const uint64_t in = kind == 0 ? h->d : h->F, outf = kind == 0 ? h->F : h->d;
+    int rc;
+    if (h->layout == MOE_LAYOUT_OUT_IN)
+        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, in, static_cast<uint64_t>(h->E) * outf,
+                       gemm_ts_kstep(), kBM);
+    else
+        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, outf, static_cast<uint64_t>(h->E) * in,
+                       kBM, kBK);
     if (rc != MOE_OK) return rc;
     if (h->wmaps.size() >= 64) h->wmaps.erase(h->wmaps.begin());
     h->wmaps.push_back(w);
@@ -354,7 +366,8 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.E = h->E;
     up.M = h->F;
     up.K = h->d;
-    up.ksteps = h->d / kBK;
+    const bool ts = h->layout == MOE_LAYOUT_OUT_IN;
+    up.ksteps = h->d / kstep_of(h);
     up.splits = 1;
     up.poff = poff;
     up.rperm = rperm;
@@ -364,19 +377,25 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.h = static_cast<__nv_bfloat16 *>(h->b_h.ptr);
     up.err = h->err;
     up.timeout_ns = h->timeout_ns;
-    if (timed(h, K_UP, s, [&] { return launch_gemm_up(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s); }) != cudaSuccess)
+    if (timed(h, K_UP, s, [&] {
+            return ts ? launch_gemm_up_ts(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s)
+                      : launch_gemm_up(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s);
+        }) != cudaSuccess)
         return MOE_ECUDA;
 
     GemmArgs dn = up;
     dn.M = h->d;
     dn.K = h->F;
     dn.splits = splits;
-    dn.ksteps = h->F / kBK / splits;
+    dn.ksteps = h->F / kstep_of(h) / splits;
     dn.s0 = static_cast<const __nv_bfloat16 *>(s_1);
     dn.s1 = nullptr;
     dn.h = nullptr;
     dn.slots = static_cast<float *>(h->b_slots.ptr);
-    if (timed(h, K_DOWN, s, [&] { return launch_gemm_down(bn, *m_w1, *m_h, dn, h->num_sms, s); }) != cudaSuccess)
+    if (timed(h, K_DOWN, s, [&] {
+            return ts ? launch_gemm_down_ts(bn, *m_w1, *m_h, dn, h->num_sms, s)
+                      : launch_gemm_down(bn, *m_w1, *m_h, dn, h->num_sms, s);
+        }) != cudaSuccess)
         return MOE_ECUDA;
 
     CombineArgs ca{T, h->d, splits, static_cast<const float *>(h->b_slots.ptr), static_cast<__nv_bfloat16 *>(out),
@@ -467,6 +486,27 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns)
     if (!h || ns < 0) return MOE_EINVAL;
     h->timeout_ns = ns;
     return MOE_OK;
+}
+
+MOE_API int moe_set_weight_layout(moe_handle h, int layout)
+{
+    if (!h || (layout != MOE_LAYOUT_IN_OUT && layout != MOE_LAYOUT_OUT_IN)) return MOE_EINVAL;
+    h->layout = layout;
+    return MOE_OK;
+}
+
+MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream)
+{
+    if (!h || !w || !w_packed || !aligned16(w) || !aligned16(w_packed)) return MOE_EINVAL;
+    if (which != 0 && which != 1) return MOE_EINVAL;
+    const size_t bytes = static_cast<size_t>(h->E) * h->d * h->F;
+    if (overlaps(w, bytes, w_packed, bytes)) return MOE_EINVAL;
+    int rc = ensure_device(h);
+    if (rc != MOE_OK) return rc;
+    const int K = which == 0 ? h->d : h->F, M = which == 0 ? h->F : h->d;
+    return launch_transpose_i8(w, w_packed, h->E, K, M, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ECUDA;
 }
 
 MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits)

@@ -29,18 +29,25 @@ def tiny_inputs():
     return inp
 
 
-@pytest.fixture(scope="module")
-def tiny_handle(m):
+LAYOUTS = [0, 1]   # MOE_LAYOUT_IN_OUT (weights through shared memory), MOE_LAYOUT_OUT_IN (through TMEM)
+
+
+@pytest.fixture(scope="module", params=LAYOUTS, ids=["in_out", "out_in"])
+def tiny_handle(m, request, tiny_inputs):
     rc, h = m.moe_create(256, 512, 8, 2)
     assert rc == 0
-    yield h
+    m.check(m.moe_set_weight_layout(h, request.param))
+    dev = parity.to_dev(tiny_inputs.layers[0])
+    if request.param == m.MOE_LAYOUT_OUT_IN:
+        dev = m.pack_layer(h, dev)
+    yield h, dev, request.param
     m.moe_destroy(h)
 
 
-def _run_tiny(m, h, inp, T, bias=None, x=None):
+def _run_tiny(m, hl, inp, T, bias=None, x=None):
+    h, dev, _ = hl
     layer_cpu = inp.layers[0]
     x_cpu = inp.x[:T] if x is None else x
-    dev = parity.to_dev(layer_cpu)
     run = parity.Run(h, x_cpu.cuda(), dev, None if bias is None else bias.cuda())
     ref = oracle.route(x_cpu, layer_cpu["router_w"], bias)
     near = parity.check_routing(run, ref, 8)
@@ -93,35 +100,50 @@ def test_tiny_token_permutation(m, tiny_inputs, tiny_handle):
 
 
 def test_forward_host_matches_device_path(m, tiny_inputs, tiny_handle):
+    h, layer, _ = tiny_handle
     T = 100
-    layer = parity.to_dev(tiny_inputs.layers[0])
     x_host = tiny_inputs.x[:T].clone().pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
-    m.check(m.moe_forward_host(tiny_handle, T, x_host, *m.layer_args(layer), out_host))
-    m.check(m.moe_sync_status(tiny_handle))
-    run = parity.Run(tiny_handle, x_host.cuda(), layer)
+    m.check(m.moe_forward_host(h, T, x_host, *m.layer_args(layer), out_host))
+    m.check(m.moe_sync_status(h))
+    run = parity.Run(h, x_host.cuda(), layer)
     assert torch.equal(out_host, run.out_h)
 
 
 def test_kernel_times_reported(m, tiny_inputs, tiny_handle):
-    layer = parity.to_dev(tiny_inputs.layers[0])
+    h, layer, _ = tiny_handle
     x = tiny_inputs.x[:64].cuda()
     out = torch.empty_like(x)
-    m.check(m.moe_set_profiling(tiny_handle, True))
+    m.check(m.moe_set_profiling(h, True))
     for _ in range(3):
-        m.check(m.moe_forward(tiny_handle, 64, x, *m.layer_args(layer), out))
-    rc, times = m.moe_get_kernel_times(tiny_handle)
-    m.check(m.moe_set_profiling(tiny_handle, False))
+        m.check(m.moe_forward(h, 64, x, *m.layer_args(layer), out))
+    rc, times = m.moe_get_kernel_times(h)
+    m.check(m.moe_set_profiling(h, False))
     assert rc == 0
     for k in ("router", "dispatch", "gather", "up_proj", "down_proj", "combine"):
         assert times[k][1] == 3 and times[k][0] > 0
 
 
+def test_pack_weight_is_a_transpose(m, tiny_handle):
+    h, _, _ = tiny_handle
+    g = torch.Generator(device="cuda").manual_seed(3)
+    w = torch.randint(-127, 128, (8, 256, 512), generator=g, device="cuda", dtype=torch.int8)
+    p = torch.empty((8, 512, 256), dtype=torch.int8, device="cuda")
+    m.check(m.moe_pack_weight(h, w, p, 0))
+    w1 = torch.randint(-127, 128, (8, 512, 256), generator=g, device="cuda", dtype=torch.int8)
+    p1 = torch.empty((8, 256, 512), dtype=torch.int8, device="cuda")
+    m.check(m.moe_pack_weight(h, w1, p1, 1))
+    torch.cuda.synchronize()
+    assert torch.equal(p, w.transpose(1, 2))
+    assert torch.equal(p1, w1.transpose(1, 2))
+
+
 def test_tiny_maximum_token_count(m, tiny_handle):
+    h, _, layout = tiny_handle
     T = m.MOE_MAX_TOKENS
     inp = moe_synth.make_inputs("tiny", device="cuda", T=T)
     layer = inp.layers[0]
-    run = parity.Run(tiny_handle, inp.x, layer)
+    run = parity.Run(h, inp.x, m.pack_layer(h, layer) if layout == m.MOE_LAYOUT_OUT_IN else layer)
     layer_cpu = parity.to_cpu(layer)
     x_cpu = inp.x.cpu()
     ref = oracle.route(x_cpu, layer_cpu["router_w"])
@@ -131,14 +153,6 @@ def test_tiny_maximum_token_count(m, tiny_handle):
 
 
 # ---- Grok-1 shape ---------------------------------------------------------------
-
-@pytest.fixture(scope="module")
-def grok_handle(m):
-    rc, h = m.moe_create(6144, 32768, 8, 2)
-    assert rc == 0
-    yield h
-    m.moe_destroy(h)
-
 
 @pytest.fixture(scope="module")
 def grok_layer():
@@ -151,8 +165,23 @@ def grok_layer():
     torch.cuda.empty_cache()
 
 
+@pytest.fixture(scope="module", params=LAYOUTS, ids=["in_out", "out_in"])
+def grok_handle(m, request, grok_layer):
+    rc, h = m.moe_create(6144, 32768, 8, 2)
+    assert rc == 0
+    m.check(m.moe_set_weight_layout(h, request.param))
+    layer = grok_layer[0]
+    if request.param == m.MOE_LAYOUT_OUT_IN:
+        layer = m.pack_layer(h, layer)
+    yield h, layer, request.param
+    m.moe_destroy(h)
+    del layer
+    torch.cuda.empty_cache()
+
+
 def test_decode_T8_all_tokens(m, grok_handle, grok_layer):
-    layer, layer_cpu = grok_layer
+    grok_handle, layer, _ = grok_handle
+    _, layer_cpu = grok_layer
     inp = moe_synth.make_inputs("decode", device="cuda")   # same seed: x drawn after the same weights
     x = inp.x
     del inp
@@ -165,7 +194,8 @@ def test_decode_T8_all_tokens(m, grok_handle, grok_layer):
 
 @pytest.mark.parametrize("name,T", [("prefill", 8192), ("skewed", 4096)])
 def test_large_T_sampled(m, grok_handle, grok_layer, name, T):
-    layer, layer_cpu = grok_layer
+    grok_handle, layer, _ = grok_handle
+    _, layer_cpu = grok_layer
     w = moe_synth.WORKLOADS[name]
     g = moe_synth.generator(w.seed + 17, "cuda")
     x = moe_synth.draw_tokens(T, w.d, g, "cuda")
@@ -184,8 +214,12 @@ def test_large_T_sampled(m, grok_handle, grok_layer, name, T):
 def test_stacked_blocks_per_block(m, grok_handle):
     """Four residual blocks, T=32: each block on the GPU is fed the oracle's residual
     stream (bf16) so that every block is compared on identical inputs."""
+    grok_handle, _, layout = grok_handle
     w = moe_synth.WORKLOADS["stacked"]
     inp = moe_synth.make_inputs("stacked", device="cuda")
+    layers_dev = inp.layers
+    if layout == m.MOE_LAYOUT_OUT_IN:
+        layers_dev = [m.pack_layer(grok_handle, l) for l in inp.layers]
     layers_cpu = [parity.to_cpu(l) for l in inp.layers]
     gam_cpu = [{k: v.cpu() for k, v in g.items()} for g in inp.gammas]
     chain = oracle.block_chain(layers_cpu, gam_cpu, inp.x.cpu(), eps=w.eps)
@@ -194,7 +228,7 @@ def test_stacked_blocks_per_block(m, grok_handle):
         h_dev = h_in.cuda().contiguous()
         m.check(m.moe_set_router_bias(grok_handle, None))
         m.check(m.moe_block_forward(grok_handle, w.T, h_dev, inp.gammas[b]["pre"], inp.gammas[b]["post"], w.eps,
-                                    *m.layer_args(inp.layers[b])))
+                                    *m.layer_args(layers_dev[b])))
         idx = torch.empty((w.T, 2), dtype=torch.int32, device="cuda")
         m.check(m.moe_get_routing(grok_handle, idx))
         m.check(m.moe_sync_status(grok_handle))
