@@ -47,8 +47,8 @@ def parse():
     p.add_argument("--tokens", type=int, default=None, help="override T")
     p.add_argument("--ffn", type=int, default=None, help="override the FFN width")
     p.add_argument("--skip-extras", action="store_true", help="skip the per-kernel and end-to-end passes")
-    p.add_argument("--layout", choices=("out_in", "in_out"), default="out_in",
-                   help="weight layout: out_in = K-major, packed once at load (TMEM path); in_out = as drawn")
+    p.add_argument("--layout", choices=("packed", "in_out"), default="packed",
+                   help="weight layout: packed = tiles written once at load (TMEM path); in_out = as drawn")
     return p.parse_args()
 
 
@@ -235,9 +235,9 @@ def run_native(args, world, rank, local):
 
     h = moe.MoELayer(w.d, w.F, w.E, w.k)
     moe.check(moe.moe_set_router_bias(h.h, bias))
-    if args.layout == "out_in":
+    if args.layout == "packed":
         # one-time weight-load step, outside every timed region: K-major int8 copies
-        moe.check(moe.moe_set_weight_layout(h.h, moe.MOE_LAYOUT_OUT_IN))
+        moe.check(moe.moe_set_weight_layout(h.h, moe.MOE_LAYOUT_PACKED))
         drawn = layers
         layers = [moe.pack_layer(h.h, l) for l in drawn]
         torch.cuda.synchronize(dev)
@@ -372,7 +372,7 @@ def run_native(args, world, rank, local):
         "config": {"workload": args.workload, "T_per_gpu": T, "d_model": w.d, "ffn": w.F, "experts": w.E,
                    "top_k": w.k, "blocks": w.blocks or 1,
                    "weights": "int8 + bf16 per-output-channel scales, layout " + args.layout +
-                              (" (packed once at load, untimed)" if args.layout == "out_in" else ""),
+                              (" (packed once at load, untimed)" if args.layout == "packed" else ""),
                    "l2": "inputs larger than L2 (%.2f GB of weights per step)" % (layer_bytes / 1e9),
                    "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],
                    "down_splits": moe.moe_plan(h.h, T)[2]},

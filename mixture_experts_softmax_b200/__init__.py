@@ -28,7 +28,7 @@ MOE_ETIMEOUT = -5
 MOE_ENODEV = -6
 MOE_MAX_TOKENS = 262144
 MOE_LAYOUT_IN_OUT = 0
-MOE_LAYOUT_OUT_IN = 1
+MOE_LAYOUT_PACKED = 1
 
 KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm")
 
@@ -184,14 +184,13 @@ def moe_pack_weight(h, w, w_packed, which: int, stream=None) -> int:
 
 
 def pack_layer(h, layer: dict, stream=None) -> dict:
-    """A copy of `layer` with its three int8 weights rewritten to MOE_LAYOUT_OUT_IN
-    (new device buffers; scales and router weight shared with `layer`)."""
+    """A copy of `layer` with its three int8 weights rewritten to MOE_LAYOUT_PACKED
+    (new flat device buffers; scales and router weight shared with `layer`)."""
     import torch
     out = dict(layer)
     for key, which in (("wl", 0), ("wv", 0), ("w1", 1)):
         w = layer[key]
-        E, a, b = w.shape
-        p = torch.empty((E, b, a), dtype=torch.int8, device=w.device)
+        p = torch.empty(w.numel(), dtype=torch.int8, device=w.device)
         check(moe_pack_weight(h, w, p, which, stream), "moe_pack_weight")
         out[key] = p
     return out

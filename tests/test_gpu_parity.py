@@ -29,16 +29,16 @@ def tiny_inputs():
     return inp
 
 
-LAYOUTS = [0, 1]   # MOE_LAYOUT_IN_OUT (weights through shared memory), MOE_LAYOUT_OUT_IN (through TMEM)
+LAYOUTS = [0, 1]   # MOE_LAYOUT_IN_OUT (weights through shared memory), MOE_LAYOUT_PACKED (packed tiles, through TMEM)
 
 
-@pytest.fixture(scope="module", params=LAYOUTS, ids=["in_out", "out_in"])
+@pytest.fixture(scope="module", params=LAYOUTS, ids=["in_out", "packed"])
 def tiny_handle(m, request, tiny_inputs):
     rc, h = m.moe_create(256, 512, 8, 2)
     assert rc == 0
     m.check(m.moe_set_weight_layout(h, request.param))
     dev = parity.to_dev(tiny_inputs.layers[0])
-    if request.param == m.MOE_LAYOUT_OUT_IN:
+    if request.param == m.MOE_LAYOUT_PACKED:
         dev = m.pack_layer(h, dev)
     yield h, dev, request.param
     m.moe_destroy(h)
@@ -124,18 +124,15 @@ def test_kernel_times_reported(m, tiny_inputs, tiny_handle):
         assert times[k][1] == 3 and times[k][0] > 0
 
 
-def test_pack_weight_is_a_transpose(m, tiny_handle):
+def test_pack_weight_layout(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
-    w = torch.randint(-127, 128, (8, 256, 512), generator=g, device="cuda", dtype=torch.int8)
-    p = torch.empty((8, 512, 256), dtype=torch.int8, device="cuda")
-    m.check(m.moe_pack_weight(h, w, p, 0))
-    w1 = torch.randint(-127, 128, (8, 512, 256), generator=g, device="cuda", dtype=torch.int8)
-    p1 = torch.empty((8, 256, 512), dtype=torch.int8, device="cuda")
-    m.check(m.moe_pack_weight(h, w1, p1, 1))
-    torch.cuda.synchronize()
-    assert torch.equal(p, w.transpose(1, 2))
-    assert torch.equal(p1, w1.transpose(1, 2))
+    for which, shape in ((0, (8, 256, 512)), (1, (8, 512, 256))):
+        w = torch.randint(-127, 128, shape, generator=g, device="cuda", dtype=torch.int8)
+        p = torch.empty(w.numel(), dtype=torch.int8, device="cuda")
+        m.check(m.moe_pack_weight(h, w, p, which))
+        torch.cuda.synchronize()
+        assert torch.equal(p, parity.packed_reference(w))
 
 
 def test_tiny_maximum_token_count(m, tiny_handle):
@@ -143,7 +140,7 @@ def test_tiny_maximum_token_count(m, tiny_handle):
     T = m.MOE_MAX_TOKENS
     inp = moe_synth.make_inputs("tiny", device="cuda", T=T)
     layer = inp.layers[0]
-    run = parity.Run(h, inp.x, m.pack_layer(h, layer) if layout == m.MOE_LAYOUT_OUT_IN else layer)
+    run = parity.Run(h, inp.x, m.pack_layer(h, layer) if layout == m.MOE_LAYOUT_PACKED else layer)
     layer_cpu = parity.to_cpu(layer)
     x_cpu = inp.x.cpu()
     ref = oracle.route(x_cpu, layer_cpu["router_w"])
@@ -165,13 +162,13 @@ def grok_layer():
     torch.cuda.empty_cache()
 
 
-@pytest.fixture(scope="module", params=LAYOUTS, ids=["in_out", "out_in"])
+@pytest.fixture(scope="module", params=LAYOUTS, ids=["in_out", "packed"])
 def grok_handle(m, request, grok_layer):
     rc, h = m.moe_create(6144, 32768, 8, 2)
     assert rc == 0
     m.check(m.moe_set_weight_layout(h, request.param))
     layer = grok_layer[0]
-    if request.param == m.MOE_LAYOUT_OUT_IN:
+    if request.param == m.MOE_LAYOUT_PACKED:
         layer = m.pack_layer(h, layer)
     yield h, layer, request.param
     m.moe_destroy(h)
@@ -218,7 +215,7 @@ def test_stacked_blocks_per_block(m, grok_handle):
     w = moe_synth.WORKLOADS["stacked"]
     inp = moe_synth.make_inputs("stacked", device="cuda")
     layers_dev = inp.layers
-    if layout == m.MOE_LAYOUT_OUT_IN:
+    if layout == m.MOE_LAYOUT_PACKED:
         layers_dev = [m.pack_layer(grok_handle, l) for l in inp.layers]
     layers_cpu = [parity.to_cpu(l) for l in inp.layers]
     gam_cpu = [{k: v.cpu() for k, v in g.items()} for g in inp.gammas]
