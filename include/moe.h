@@ -65,7 +65,7 @@ extern "C" {
 
 /* Weight layouts (moe_set_weight_layout). */
 #define MOE_LAYOUT_IN_OUT 0   /* w_lin, w_v [E, d, F]; w_1 [E, F, d]  (x @ W orientation, default) */
-#define MOE_LAYOUT_PACKED 1   /* 16 KB tiles written by moe_pack_weight (see there)               */
+#define MOE_LAYOUT_PACKED 1   /* w_lin, w_v [E, F, d]; w_1 [E, d, F]  (input dim contiguous)      */
 
 typedef struct moe_ctx *moe_handle;
 
@@ -184,28 +184,24 @@ MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
 
 /*
  * Select how the forward calls of this handle read w_lin, w_v and w_1:
- *   MOE_LAYOUT_IN_OUT (default)  the [E, in, out] layout of the block above;
- *   MOE_LAYOUT_PACKED            the tile layout written by moe_pack_weight.
+ *   MOE_LAYOUT_IN_OUT (default)  [E, in, out]: the layout block above;
+ *   MOE_LAYOUT_PACKED            [E, out, in]: each output feature's input
+ *                                elements contiguous (w_lin, w_v [E, F, d];
+ *                                w_1 [E, d, F]); written by moe_pack_weight.
  * Both give the same result up to fp32 summation order.  With MOE_LAYOUT_PACKED
- * the GEMMs stream each weight tile with one contiguous copy and keep the
- * dequantised bf16 weights in tensor memory instead of shared memory: the fast
- * path.  Repacking is a one-time cost at weight-load time.  Scales are the same
- * in both layouts.  Returns MOE_EINVAL for an unknown layout.
+ * the GEMMs keep the dequantised bf16 weights in tensor memory instead of shared
+ * memory: the fast path.  The layout change is a one-time cost at weight-load
+ * time.  Scales are the same in both layouts.  Returns MOE_EINVAL for an
+ * unknown layout.
  */
 MOE_API int moe_set_weight_layout(moe_handle h, int layout);
 
 /*
- * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT into MOE_LAYOUT_PACKED
- * (values copied unchanged), enqueued on `stream`.
- *   which = 0: w is linear or linear_v, [E, in = d, out = F]
- *   which = 1: w is linear_1,           [E, in = F, out = d]
+ * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT to MOE_LAYOUT_PACKED
+ * (a per-expert transpose; values copied unchanged), enqueued on `stream`.
+ *   which = 0: w is linear or linear_v, [E, d, F] -> w_packed [E, F, d]
+ *   which = 1: w is linear_1,           [E, F, d] -> w_packed [E, d, F]
  * w and w_packed are device buffers of E*d*F bytes that must not overlap.
- * Packed layout, with K = in, M = out: one 16 KB tile per (expert e, block
- * mt = o / 128 of output features, block kt = i / 128 of input elements), at
- * byte offset ((e * M/128 + mt) * K/128 + kt) * 16384; inside the tile, output
- * feature r = o % 128 owns bytes [128 r, 128 r + 128), which hold its 128 input
- * elements in 16-byte chunks, chunk c = (i % 128) / 16 stored at chunk c ^ (r % 8):
- *   w_packed[tile + 128 r + 16 (c ^ (r % 8)) + i % 16] = w[e, i, o].
  */
 MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream);
 

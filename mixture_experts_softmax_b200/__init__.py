@@ -185,12 +185,13 @@ def moe_pack_weight(h, w, w_packed, which: int, stream=None) -> int:
 
 def pack_layer(h, layer: dict, stream=None) -> dict:
     """A copy of `layer` with its three int8 weights rewritten to MOE_LAYOUT_PACKED
-    (new flat device buffers; scales and router weight shared with `layer`)."""
+    (new device buffers; scales and router weight shared with `layer`)."""
     import torch
     out = dict(layer)
     for key, which in (("wl", 0), ("wv", 0), ("w1", 1)):
         w = layer[key]
-        p = torch.empty(w.numel(), dtype=torch.int8, device=w.device)
+        E, a, b = w.shape
+        p = torch.empty((E, b, a), dtype=torch.int8, device=w.device)
         check(moe_pack_weight(h, w, p, which, stream), "moe_pack_weight")
         out[key] = p
     return out

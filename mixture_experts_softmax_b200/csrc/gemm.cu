@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 16) {
                     float va[16], vb[16];
+                    __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
                     tmem_ld16(tl + c, va);
                     tmem_ld16(tl + BN + c, vb);
                     tmem_wait_ld();
@@ -268,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 16) {
                     float v[16];
+                    __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
                     tmem_ld16(tl + c, v);
                     tmem_wait_ld();
 #pragma unroll

@@ -1,6 +1,6 @@
-// gemm_ts.cu -- grouped expert GEMMs for int8 weights in the packed tile layout (see
-// pack.cu), with the dequantised bf16 weights kept in tensor memory (TMEM) as the
-// MMA's A operand.
+// gemm_ts.cu -- grouped expert GEMMs for int8 weights stored K-major ([E, out, in], one
+// row of reduction elements per output feature), with the dequantised bf16 weights
+// kept in tensor memory (TMEM) as the MMA's A operand.
 //
 // Computes the expert MLP of "Grok-1 Admin & Architecture Guide", section 3,
 // "Mixture of Experts (MoELayer + Router)" step 3, linear_1(gelu(linear(x)) * linear_v(x)),
@@ -9,15 +9,12 @@
 // Same tile orientation as the shared-memory variant (weights = A, M = 128 output
 // features; grouped token rows = B, N = BN rows), but per pipeline stage of 128
 // reduction elements:
-//   - a producer thread copies the int8 weight tile(s) [128 f x 128 k], each a
-//     contiguous, already swizzled 16 KB block of the packed layout, into a
-//     shared-memory staging ring with 1-D bulk copies (full DRAM bursts);
-//   - 16 converter warps in G groups of 4 * (matrices per stage) warps: group g takes
-//     every G-th stage, each warp owns 32 feature rows (one TMEM lane quadrant) of one
-//     matrix and each thread a whole 128-byte row; it converts int8 -> bf16 exactly
-//     and stores the bf16 pairs into the A ring in TMEM with tcgen05.st (one 32-bit
-//     TMEM column holds two consecutive k).  While one group waits on its stores and
-//     barriers, the other groups convert;
+//   - a TMA producer thread copies the int8 weight tile(s) [128 f x 128 k] (128-byte
+//     swizzle) into a shared-memory staging ring;
+//   - 16 converter warps each own 32 feature rows (one TMEM lane quadrant) and a slice
+//     of the 128 reduction elements: they read their bytes from the staging tile,
+//     convert int8 -> bf16 exactly and store the bf16 pairs into the A ring in TMEM
+//     with tcgen05.st (one 32-bit TMEM column holds two consecutive k);
 //   - a second TMA producer copies the bf16 activation tile [BN r x 128 k] into the
 //     shared-memory operand ring;
 //   - one thread issues tcgen05.mma with A from TMEM and B from shared memory;
@@ -40,13 +37,11 @@ constexpr int kBKT = 128;                      // reduction elements per stage
 constexpr int kSmemBudget = 208 * 1024;
 static_assert(kWarpConv0 % 4 == 0, "converter warp w must own TMEM lane quadrant w % 4");
 
-constexpr int kTileBytes = kBM * kBKT;         // one packed weight tile
-
 template <bool UP, int BN>
 struct CfgTS {
     static constexpr int NA = UP ? 2 : 1;                   // weight matrices per stage
-    static constexpr int NG = 4 * NA;                       // converter warps per stage group
-    static constexpr int G = kConvWarps / NG;               // stage groups
+    static constexpr int KP = kConvWarps / 4 / NA;          // converter warps per (quadrant, matrix)
+    static constexpr int CH = (kBKT / 16) / KP;             // 16-byte chunks per converter thread and stage
     static constexpr int STG = NA * kBM * kBKT;             // int8 staging bytes per stage
     static constexpr int BBYTES = BN * kBKT * 2;            // bf16 activation bytes per stage
     static constexpr int NDB = (UP && BN == 128) ? 1 : 2;   // accumulator buffers in TMEM
@@ -67,7 +62,7 @@ struct CfgTS {
     static_assert(S1 >= 2 && S2 >= 2, "rings too shallow");
     static_assert(SMEM <= 227 * 1024, "shared memory over the per-CTA limit");
     static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
-    static_assert(G * NG == kConvWarps, "converter warps split evenly into stage groups");
+    static_assert(CH * 8 == 16 || CH * 8 == 32, "a converter thread stores 16 or 32 TMEM columns");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is 16..256 in steps of 16");
 };
 
@@ -80,7 +75,9 @@ __device__ __forceinline__ constexpr uint32_t idesc_ts()
 }
 
 template <bool UP, int BN>
-__global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_constant__ CUtensorMap tmB, const GemmArgs a)
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_ts_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, const GemmArgs a)
 {
     using C = CfgTS<UP, BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -107,10 +104,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::S1; ++s) {
             mbar_init(stg_full(s), 1);
-            mbar_init(stg_empty(s), C::NG);
+            mbar_init(stg_empty(s), kConvWarps);
         }
         for (int s = 0; s < C::S2; ++s) {
-            mbar_init(a_full(s), C::NG);
+            mbar_init(a_full(s), kConvWarps);
             mbar_init(b_full(s), 1);
             mbar_init(op_empty(s), 1);
         }
@@ -130,7 +127,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
         tmem_alloc(smem_u32(misc), C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == kWarpTmaA && lane == 0) prefetch_tmap(&tmB);
+    if (warp == kWarpTmaA && lane == 0) {
+        prefetch_tmap(&tmA0);
+        if (UP) prefetch_tmap(&tmA1);
+        prefetch_tmap(&tmB);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -142,22 +143,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
     const Waiter w{abort_flag, a.err, a.timeout_ns, UP ? 20 : 40};
 
     if (warp == kWarpTmaA) {
-        // ---- packed int8 weight tiles (16 KB each) -> staging ring ----------------------
+        // ---- int8 weight tiles [128 f x 128 k] -> staging ring ------------------------
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
-            const int kt = a.K / kBKT;
             uint32_t st = 0, ph = 0, issued = 0, par = 0;
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
                 int e, m, n, s;
                 decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
-                const size_t t0 = ((static_cast<size_t>(e) * m_tiles + m) * kt + s * a.ksteps) * kTileBytes;
+                const int kb = s * a.ksteps;
+                const int y = e * a.M + m * kBM;
                 for (int ks = 0; ks < a.ksteps; ++ks) {
                     if (!w.wait(stg_empty(st), ph ^ 1u, 1)) goto a_done;
                     mbar_arrive_expect_tx(stg_full(st), C::STG);
                     const uint32_t dst = sbase + C::OFF_STG + st * C::STG;
-                    const size_t off = t0 + static_cast<size_t>(ks) * kTileBytes;
-                    bulk_load(dst, a.wa0 + off, kTileBytes, stg_full(st), pol);
-                    if (UP) bulk_load(dst + kTileBytes, a.wa1 + off, kTileBytes, stg_full(st), pol);
+                    tma_load_2d(dst, &tmA0, stg_full(st), (kb + ks) * kBKT, y, pol);
+                    if (UP) tma_load_2d(dst + kBM * kBKT, &tmA1, stg_full(st), (kb + ks) * kBKT, y, pol);
                     issued |= 1u << st;
                     par = (par & ~(1u << st)) | (ph << st);
                     if (++st == C::S1) { st = 0; ph ^= 1u; }
@@ -210,9 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
                 bool ok = true;
                 for (int ks = 0; ks < a.ksteps; ++ks) {
                     if (!w.wait(a_full(st), ph, 4) || !w.wait(b_full(st), ph, 5)) { ok = false; break; }
-#ifdef MOE_PIPE_STATS
-                    const long long q0 = clock64();
-#endif
                     tc_fence_after();
                     const uint32_t acol = tmem_base + C::A_BASE + st * C::A_COLS;
                     const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
@@ -225,9 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
                                          (ks | kk) != 0);
                     }
                     umma_commit(op_empty(st));
-#ifdef MOE_PIPE_STATS
-                    atomicAdd(&g_pipe_stats[w.stat_base + 12], static_cast<unsigned long long>(clock64() - q0));
-#endif
                     if (++st == C::S2) { st = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
@@ -248,9 +242,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
             const uint32_t aph = (it / C::NDB) & 1;
             const bool ok = __all_sync(0xffffffffu, w.wait(acc_full(b), aph, 6));
             if (!ok) break;
-#ifdef MOE_PIPE_STATS
-            const long long r0 = clock64();
-#endif
             tc_fence_after();
             const int f = m * kBM + ew * 32 + lane;
             const uint32_t tl = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * C::ACC;
@@ -261,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 16) {
                     float va[16], vb[16];
+                    __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
                     tmem_ld16(tl + c, va);
                     tmem_ld16(tl + BN + c, vb);
                     tmem_wait_ld();
@@ -277,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 16) {
                     float v[16];
+                    __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
                     tmem_ld16(tl + c, v);
                     tmem_wait_ld();
 #pragma unroll
@@ -294,78 +287,62 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty(b));
-#ifdef MOE_PIPE_STATS
-            if (lane == 0) atomicAdd(&g_pipe_stats[w.stat_base + 13], static_cast<unsigned long long>(clock64() - r0));
-#endif
         }
     } else if (warp >= kWarpConv0) {
         // ---- int8 staging -> bf16 A operand in TMEM ------------------------------------
-        // Converter warp cw belongs to stage group g = cw / NG and converts the stages
-        // whose global index i (counted over this CTA's tiles) has i % G == g.  It owns
-        // TMEM lane quadrant q = warp % 4 (feature rows 32q..32q+31 of the tile) of
-        // weight matrix `mat`; each thread converts its whole 128-byte feature row.
-        // Lanes of one 8-lane phase read 8 different rows, whose swizzle puts the same
-        // logical chunk in 8 different bank groups.
+        // Converter warp cw owns TMEM lane quadrant q = warp % 4 (feature rows 32q..32q+31
+        // of the tile), weight matrix `mat` and chunks [j0, j0 + CH) of the 8 16-byte
+        // chunks of each 128-byte feature row.  Lanes of one 8-lane phase read 8
+        // different rows, whose 128-byte swizzle puts the same logical chunk in 8
+        // different bank groups.
         const int cw = warp - kWarpConv0;
-        const int g = cw / C::NG;
         const int q = warp & 3;
-        const int mat = (cw % C::NG) >> 2;
+        const int part = cw >> 2;
+        const int mat = part / C::KP;
+        const int j0 = (part % C::KP) * C::CH;
         const int fr = q * 32 + lane;
-        const uint32_t src_row = mat * kTileBytes + fr * 128;
+        const uint32_t src_row = mat * kBM * kBKT + fr * 128;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        const int my_tiles = total > static_cast<int>(blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-        const int n_stages = my_tiles * a.ksteps;
-        for (int i = g; i < n_stages; i += C::G) {
-            const int st = i % C::S1, st2 = i % C::S2;
-            const uint32_t ph = (i / C::S1) & 1u, ph2 = (i / C::S2) & 1u;
-            const bool ok = __all_sync(0xffffffffu, w.wait(stg_full(st), ph, 7) && w.wait(op_empty(st2), ph2 ^ 1u, 8));
-            if (!ok) break;
-#ifdef MOE_PIPE_STATS
-            const long long p1 = clock64();
-#endif
-            tc_fence_after();
-            const uint32_t src = sbase + C::OFF_STG + st * C::STG + src_row;
-            uint4 v[8];
+        uint32_t st = 0, ph = 0, st2 = 0, ph2 = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            bool ok = true;
+            for (int ks = 0; ks < a.ksteps; ++ks) {
+                ok = __all_sync(0xffffffffu, w.wait(stg_full(st), ph, 7) && w.wait(op_empty(st2), ph2 ^ 1u, 8));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t src = sbase + C::OFF_STG + st * C::STG + src_row;
+                uint4 v[C::CH];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = lds128(src + ((j ^ (fr & 7)) << 4));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(stg_empty(st));   // release orders the reads above before it
-            const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + mat * (kBKT / 2);
+                for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
+                uint32_t words[C::CH * 8];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t words[32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 &u = v[half * 4 + c];
-                    words[c * 8 + 0] = i8x2_to_bf16x2(u.x, 0x4140);
-                    words[c * 8 + 1] = i8x2_to_bf16x2(u.x, 0x4342);
-                    words[c * 8 + 2] = i8x2_to_bf16x2(u.y, 0x4140);
-                    words[c * 8 + 3] = i8x2_to_bf16x2(u.y, 0x4342);
-                    words[c * 8 + 4] = i8x2_to_bf16x2(u.z, 0x4140);
-                    words[c * 8 + 5] = i8x2_to_bf16x2(u.z, 0x4342);
-                    words[c * 8 + 6] = i8x2_to_bf16x2(u.w, 0x4140);
-                    words[c * 8 + 7] = i8x2_to_bf16x2(u.w, 0x4342);
+                for (int c = 0; c < C::CH; ++c) {
+                    words[c * 8 + 0] = i8x2_to_bf16x2(v[c].x, 0x4140);
+                    words[c * 8 + 1] = i8x2_to_bf16x2(v[c].x, 0x4342);
+                    words[c * 8 + 2] = i8x2_to_bf16x2(v[c].y, 0x4140);
+                    words[c * 8 + 3] = i8x2_to_bf16x2(v[c].y, 0x4342);
+                    words[c * 8 + 4] = i8x2_to_bf16x2(v[c].z, 0x4140);
+                    words[c * 8 + 5] = i8x2_to_bf16x2(v[c].z, 0x4342);
+                    words[c * 8 + 6] = i8x2_to_bf16x2(v[c].w, 0x4140);
+                    words[c * 8 + 7] = i8x2_to_bf16x2(v[c].w, 0x4342);
                 }
-                tmem_st32(taddr + half * 32, words);
+                const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + mat * (kBKT / 2) + j0 * 8;
+                __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
+                if constexpr (C::CH * 8 == 32)
+                    tmem_st32(taddr, words);
+                else
+                    tmem_st16(taddr, words);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(stg_empty(st));
+                    mbar_arrive(a_full(st2));
+                }
+                if (++st == C::S1) { st = 0; ph ^= 1u; }
+                if (++st2 == C::S2) { st2 = 0; ph2 ^= 1u; }
             }
-#ifdef MOE_PIPE_STATS
-            const long long p3 = clock64();
-#endif
-            tmem_wait_st();
-#ifdef MOE_PIPE_STATS
-            const long long p4 = clock64();
-#endif
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(a_full(st2));
-#ifdef MOE_PIPE_STATS
-                const long long p5 = clock64();
-                atomicAdd(&g_pipe_stats[w.stat_base + 9], static_cast<unsigned long long>(p3 - p1));
-                atomicAdd(&g_pipe_stats[w.stat_base + 10], static_cast<unsigned long long>(p4 - p3));
-                atomicAdd(&g_pipe_stats[w.stat_base + 11], static_cast<unsigned long long>(p5 - p4));
-#endif
-            }
+            if (!ok) break;
         }
     }
 
@@ -381,7 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(const __grid_const
 }
 
 template <bool UP, int BN>
-cudaError_t launch_one_ts(const CUtensorMap &b, const GemmArgs &args, int grid, cudaStream_t s)
+cudaError_t launch_one_ts(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b, const GemmArgs &args,
+                          int grid, cudaStream_t s)
 {
     using C = CfgTS<UP, BN>;
     static bool configured = false;   // the attribute is the same for every launch in the process
@@ -391,7 +369,7 @@ cudaError_t launch_one_ts(const CUtensorMap &b, const GemmArgs &args, int grid, 
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    gemm_ts_kernel<UP, BN><<<grid, kThreads, C::SMEM, s>>>(b, args);
+    gemm_ts_kernel<UP, BN><<<grid, kThreads, C::SMEM, s>>>(a0, a1, b, args);
     return cudaGetLastError();
 }
 
@@ -399,24 +377,26 @@ cudaError_t launch_one_ts(const CUtensorMap &b, const GemmArgs &args, int grid, 
 
 int gemm_ts_kstep() { return kBKT; }
 
-cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &xp, const GemmArgs &a, int grid, cudaStream_t s)
+cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
+                              const GemmArgs &a, int grid, cudaStream_t s)
 {
     switch (bn) {
-    case 16: return launch_one_ts<true, 16>(xp, a, grid, s);
-    case 32: return launch_one_ts<true, 32>(xp, a, grid, s);
-    case 64: return launch_one_ts<true, 64>(xp, a, grid, s);
-    case 128: return launch_one_ts<true, 128>(xp, a, grid, s);
+    case 16: return launch_one_ts<true, 16>(wl, wv, xp, a, grid, s);
+    case 32: return launch_one_ts<true, 32>(wl, wv, xp, a, grid, s);
+    case 64: return launch_one_ts<true, 64>(wl, wv, xp, a, grid, s);
+    case 128: return launch_one_ts<true, 128>(wl, wv, xp, a, grid, s);
     default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &h, const GemmArgs &a, int grid, cudaStream_t s)
+cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a, int grid,
+                                cudaStream_t s)
 {
     switch (bn) {
-    case 16: return launch_one_ts<false, 16>(h, a, grid, s);
-    case 32: return launch_one_ts<false, 32>(h, a, grid, s);
-    case 64: return launch_one_ts<false, 64>(h, a, grid, s);
-    case 128: return launch_one_ts<false, 128>(h, a, grid, s);
+    case 16: return launch_one_ts<false, 16>(w1, w1, h, a, grid, s);
+    case 32: return launch_one_ts<false, 32>(w1, w1, h, a, grid, s);
+    case 64: return launch_one_ts<false, 64>(w1, w1, h, a, grid, s);
+    case 128: return launch_one_ts<false, 128>(w1, w1, h, a, grid, s);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -65,8 +65,6 @@ struct GemmArgs {
     float *slots;               // DOWN output [splits, T, 2, M]
     int *err;                   // device error word
     long long timeout_ns;
-    const int8_t *wa0;          // packed-tile weights (tiled layout only): linear or linear_1
-    const int8_t *wa1;          // packed-tile weights: linear_v (UP only)
 };
 
 struct CombineArgs {
@@ -94,14 +92,14 @@ cudaError_t launch_gemm_up(int bn, const CUtensorMap &wl, const CUtensorMap &wv,
                            const GemmArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_gemm_down(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,
                              int grid, cudaStream_t s);
-// the same GEMMs for weights in the packed tile layout (a.wa0 / a.wa1), dequantised into TMEM
-cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &xp, const GemmArgs &a, int grid, cudaStream_t s);
-cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &h, const GemmArgs &a, int grid, cudaStream_t s);
+// the same GEMMs for K-major ([E, out, in]) weights, dequantised into TMEM
+cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
+                              const GemmArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,
+                                int grid, cudaStream_t s);
 int gemm_ts_kstep();   // reduction elements per pipeline stage of the TMEM-operand GEMMs
-// E int8 [K, M] matrices (x @ W orientation) -> packed tiles (K, M multiples of 128):
-// tile (e, M/128 block mt, K/128 block kt) is 16 KB at ((e * M/128 + mt) * K/128 + kt) * 16384; inside it
-// output feature row r (128 bytes) holds the 128 reduction elements, 16-byte chunk j at chunk j ^ (r % 8)
-cudaError_t launch_pack_tiles(const int8_t *in, int8_t *out, int E, int K, int M, cudaStream_t s);
+// out[e, m, k] = in[e, k, m] for E int8 [K, M] matrices (K, M multiples of 64)
+cudaError_t launch_transpose_i8(const int8_t *in, int8_t *out, int E, int K, int M, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_prenorm(const NormArgs &a, cudaStream_t s);
 

@@ -231,8 +231,8 @@ int encode_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *ptr
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ECUDA;
 }
 
-// int8 weight descriptor of the [E, in, out] layout: rows = E*in, box = 64 k-rows x 128 features.
-// (The packed layout is read with 1-D bulk copies and needs none.)
+// int8 weight descriptor.  [E, in, out] layout: rows = E*in, box = 64 k-rows x 128 features.
+// [E, out, in] (packed) layout: rows = E*out, box = 128 feature-rows x 128 k.
 int weight_map(moe_ctx *h, const void *ptr, int kind, const CUtensorMap **out)
 {
     for (auto &w : h->wmaps)
@@ -245,7 +245,12 @@ int weight_map(moe_ctx *h, const void *ptr, int kind, const CUtensorMap **out)
     w.kind = kind;
     w.layout = h->layout;
     const uint64_t in = kind == 0 ? h->d : h->F, outf = kind == 0 ? h->F : h->d;
-    int rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, outf, static_cast<uint64_t>(h->E) * in,
+    int rc;
+    if (h->layout == MOE_LAYOUT_PACKED)
+        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, in, static_cast<uint64_t>(h->E) * outf,
+                       gemm_ts_kstep(), kBM);
+    else
+        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, outf, static_cast<uint64_t>(h->E) * in,
                        kBM, kBK);
     if (rc != MOE_OK) return rc;
     if (h->wmaps.size() >= 64) h->wmaps.erase(h->wmaps.begin());
@@ -341,12 +346,10 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     const int rows = rows_for(h, T, bn);
 
     const bool ts = h->layout == MOE_LAYOUT_PACKED;
-    const CUtensorMap *m_wl = nullptr, *m_wv = nullptr, *m_w1 = nullptr, *m_xp, *m_h;
-    if (!ts) {
-        if ((rc = weight_map(h, w_lin, 0, &m_wl)) != MOE_OK) return rc;
-        if ((rc = weight_map(h, w_v, 0, &m_wv)) != MOE_OK) return rc;
-        if ((rc = weight_map(h, w_1, 1, &m_w1)) != MOE_OK) return rc;
-    }
+    const CUtensorMap *m_wl, *m_wv, *m_w1, *m_xp, *m_h;
+    if ((rc = weight_map(h, w_lin, 0, &m_wl)) != MOE_OK) return rc;
+    if ((rc = weight_map(h, w_v, 0, &m_wv)) != MOE_OK) return rc;
+    if ((rc = weight_map(h, w_1, 1, &m_w1)) != MOE_OK) return rc;
     if ((rc = act_maps(h, bn, &m_xp, &m_h)) != MOE_OK) return rc;
 
     RouteArgs ra{T, h->d, static_cast<const __nv_bfloat16 *>(x), router_w, h->bias, idx, gate};
@@ -365,8 +368,6 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.M = h->F;
     up.K = h->d;
     up.ksteps = h->d / kstep_of(h);
-    up.wa0 = w_lin;
-    up.wa1 = w_v;
     up.splits = 1;
     up.poff = poff;
     up.rperm = rperm;
@@ -377,7 +378,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.err = h->err;
     up.timeout_ns = h->timeout_ns;
     if (timed(h, K_UP, s, [&] {
-            return ts ? launch_gemm_up_ts(bn, *m_xp, up, h->num_sms, s)
+            return ts ? launch_gemm_up_ts(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s)
                       : launch_gemm_up(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s);
         }) != cudaSuccess)
         return MOE_ECUDA;
@@ -387,14 +388,12 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     dn.K = h->F;
     dn.splits = splits;
     dn.ksteps = h->F / kstep_of(h) / splits;
-    dn.wa0 = w_1;
-    dn.wa1 = nullptr;
     dn.s0 = static_cast<const __nv_bfloat16 *>(s_1);
     dn.s1 = nullptr;
     dn.h = nullptr;
     dn.slots = static_cast<float *>(h->b_slots.ptr);
     if (timed(h, K_DOWN, s, [&] {
-            return ts ? launch_gemm_down_ts(bn, *m_h, dn, h->num_sms, s)
+            return ts ? launch_gemm_down_ts(bn, *m_w1, *m_h, dn, h->num_sms, s)
                       : launch_gemm_down(bn, *m_w1, *m_h, dn, h->num_sms, s);
         }) != cudaSuccess)
         return MOE_ECUDA;
@@ -505,7 +504,7 @@ MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int
     int rc = ensure_device(h);
     if (rc != MOE_OK) return rc;
     const int K = which == 0 ? h->d : h->F, M = which == 0 ? h->F : h->d;
-    return launch_pack_tiles(w, w_packed, h->E, K, M, static_cast<cudaStream_t>(stream)) == cudaSuccess
+    return launch_transpose_i8(w, w_packed, h->E, K, M, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? MOE_OK
                : MOE_ECUDA;
 }

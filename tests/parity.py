@@ -98,14 +98,3 @@ def check_output(run: Run, layer_cpu: dict, x_cpu, tokens, near, bias_cpu=None, 
     assert err <= OUT_RTOL * scale, f"max|gpu-oracle| = {err:.3e} > {OUT_RTOL} * {scale:.3e}"
     return err / max(scale, 1e-300)
 
-
-def packed_reference(w):
-    """The packed tile layout of include/moe.h, built with torch indexing."""
-    E, K, M = w.shape
-    t = w.reshape(E, K // 128, 128, M // 128, 128)          # [e, kt, i%128, mt, o%128]
-    t = t.permute(0, 3, 1, 4, 2)                            # [e, mt, kt, r, i%128]
-    t = t.reshape(E, M // 128, K // 128, 128, 8, 16)        # chunks c of 16 input elements
-    r = torch.arange(128, device=w.device)
-    src_chunk = torch.arange(8, device=w.device)[None, :] ^ (r[:, None] % 8)   # stored chunk j holds c = j ^ (r % 8)
-    t = t[:, :, :, r[:, None], src_chunk, :]
-    return t.reshape(-1)

@@ -116,21 +116,3 @@ def test_forward_without_gpu_reports_no_device(m):
     finally:
         m.moe_destroy(h)
 
-
-def test_packed_reference_matches_header_formula():
-    """The torch reference of the packed tile layout equals the scalar formula of
-    include/moe.h (checked element by element on a small tensor)."""
-    import torch
-    from tests import parity
-    E, K, M = 2, 256, 384
-    g = torch.Generator().manual_seed(1)
-    w = torch.randint(-127, 128, (E, K, M), generator=g, dtype=torch.int8)
-    p = parity.packed_reference(w)
-    ref = torch.empty_like(p)
-    for e in range(E):
-        for i in range(K):
-            for o in range(M):
-                mt, kt, r, c = o // 128, i // 128, o % 128, (i % 128) // 16
-                tile = ((e * (M // 128) + mt) * (K // 128) + kt) * 16384
-                ref[tile + 128 * r + 16 * (c ^ (r % 8)) + i % 16] = w[e, i, o]
-    assert torch.equal(p, ref)

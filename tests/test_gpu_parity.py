@@ -124,15 +124,15 @@ def test_kernel_times_reported(m, tiny_inputs, tiny_handle):
         assert times[k][1] == 3 and times[k][0] > 0
 
 
-def test_pack_weight_layout(m, tiny_handle):
+def test_pack_weight_is_a_transpose(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
     for which, shape in ((0, (8, 256, 512)), (1, (8, 512, 256))):
         w = torch.randint(-127, 128, shape, generator=g, device="cuda", dtype=torch.int8)
-        p = torch.empty(w.numel(), dtype=torch.int8, device="cuda")
+        p = torch.empty((shape[0], shape[2], shape[1]), dtype=torch.int8, device="cuda")
         m.check(m.moe_pack_weight(h, w, p, which))
         torch.cuda.synchronize()
-        assert torch.equal(p, parity.packed_reference(w))
+        assert torch.equal(p, w.transpose(1, 2))
 
 
 def test_tiny_maximum_token_count(m, tiny_handle):
