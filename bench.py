@@ -94,6 +94,13 @@ def barrier(world: int, device=None):
             dist.barrier()
 
 
+def job_value(tokens_per_rank: int, world: int, ms_per_rank: float, device=None):
+    """Whole-job throughput of `world` replicas: all ranks' tokens over the slowest rank's
+    time per step.  Returns (tokens/s, slowest ms per step); every rank gets the same pair."""
+    ms_max = max_over_ranks(ms_per_rank, world, device)
+    return tokens_per_rank * world / (ms_max / 1e3), ms_max
+
+
 def dist_teardown(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -283,9 +290,8 @@ def run_native(args, world, rank, local):
     ms = e0.elapsed_time(e1) / K
     clk = clocks.stop() if clocks else None
     moe.check(moe.moe_sync_status(h.h, stream), "device status after the timed region")
-    ms_max = max_over_ranks(ms, world, dev)
+    value, ms_max = job_value(T, world, ms, dev)
     tokens = T * world
-    value = tokens / (ms_max / 1e3)
 
     if args.skip_extras:
         h.close()
