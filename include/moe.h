@@ -211,6 +211,36 @@ MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int
  */
 MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits);
 
+/* Largest token count moe_route_noalloc accepts (its static scratch is sized for it). */
+#define MOE_NOALLOC_MAX_TOKENS 65536
+
+/*
+ * Routing only -- router (fp32 logits, softmax, top-2) and dispatch (grouping by
+ * expert) -- without allocating any device memory.  The pages have no counterpart:
+ * this entry point exists for callers that cannot call cudaMalloc, such as code
+ * running inside a device-memory arena that is sized once up front, or code inside
+ * a framework that owns the allocator.  It needs no handle.
+ *   x         bf16 [T, d] input tokens (d a multiple of 8)
+ *   router_w  fp32 [d, 8]
+ *   bias      fp32 [8] added to the logits, or NULL
+ *   idx       int32 [T, 2], gate fp32 [T, 2], offsets int32 [9], perm int32 [2T]:
+ *             outputs with the meaning of moe_get_routing (E = 8 experts)
+ * All pointers are device pointers, 16-byte aligned, owned by the caller.
+ * Scratch: dispatch's working arrays live in one file-scope device array of about
+ * 1 MB (MOE_NOALLOC_MAX_TOKENS tokens), which every GPU that loads the library holds
+ * until the process exits.  The first call on a device looks up that array's device
+ * address (cudaGetSymbolAddress, with the device current); make that first call
+ * before any stream capture.  Every call shares the array and it keeps the last
+ * call's contents; each call writes every word it later reads, so nothing needs
+ * clearing, but calls whose kernels overlap on the GPU (different streams, or
+ * concurrent host threads) race on it: serialise them.
+ * Returns MOE_EINVAL for T > MOE_NOALLOC_MAX_TOKENS, a bad d, or a null or
+ * misaligned pointer; MOE_ENODEV without a device; MOE_ECUDA if a launch failed.
+ * Calls no allocating routine.  T == 0 is a no-op.
+ */
+MOE_API int moe_route_noalloc(int T, int d, const void *x, const float *router_w, const float *bias,
+                              int32_t *idx, float *gate, int32_t *offsets, int32_t *perm, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

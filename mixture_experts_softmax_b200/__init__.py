@@ -29,6 +29,7 @@ MOE_ENODEV = -6
 MOE_MAX_TOKENS = 262144
 MOE_LAYOUT_IN_OUT = 0
 MOE_LAYOUT_PACKED = 1
+MOE_NOALLOC_MAX_TOKENS = 65536
 
 KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm")
 
@@ -37,7 +38,7 @@ EXPORTS = (
     "moe_strerror", "moe_version", "moe_create", "moe_destroy", "moe_set_router_bias",
     "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing",
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
-    "moe_set_weight_layout", "moe_pack_weight",
+    "moe_set_weight_layout", "moe_pack_weight", "moe_route_noalloc",
 )
 
 
@@ -71,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "moe_plan": (I, [P, I, ctypes.POINTER(I), ctypes.POINTER(I)]),
         "moe_set_weight_layout": (I, [P, I]),
         "moe_pack_weight": (I, [P, P, P, I, P]),
+        "moe_route_noalloc": (I, [I, I, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -195,6 +197,11 @@ def pack_layer(h, layer: dict, stream=None) -> dict:
         check(moe_pack_weight(h, w, p, which, stream), "moe_pack_weight")
         out[key] = p
     return out
+
+
+def moe_route_noalloc(T, d, x, router_w, bias, idx, gate, offsets, perm, stream=None) -> int:
+    return _lib.moe_route_noalloc(int(T), int(d), _ptr(x), _ptr(router_w), _ptr(bias), _ptr(idx), _ptr(gate),
+                                  _ptr(offsets), _ptr(perm), _stream(stream))
 
 
 def moe_plan(h, T: int):
