@@ -37,16 +37,23 @@ constexpr int kBKT = 128;                      // reduction elements per stage
 constexpr int kSmemBudget = 208 * 1024;
 static_assert(kWarpConv0 % 4 == 0, "converter warp w must own TMEM lane quadrant w % 4");
 
+// Weight tiles are [128 features x 128 reduction elements] int8 "boxes" of 16 KB.  A pipeline
+// stage carries NB boxes: the up-projection one box of each of its two matrices (same k), the
+// down-projection with narrow tiles two consecutive k-boxes of its one matrix (so every stage
+// moves 32 KB), the down-projection with 128-route tiles one box.
 template <bool UP, int BN>
 struct CfgTS {
-    static constexpr int NA = UP ? 2 : 1;                   // weight matrices per stage
-    static constexpr int KP = kConvWarps / 4 / NA;          // converter warps per (quadrant, matrix)
+    static constexpr int NA = UP ? 2 : 1;                   // weight matrices = accumulators
+    static constexpr bool K2 = !UP && BN <= 64;             // two k-boxes per stage
+    static constexpr int NB = UP ? 2 : (K2 ? 2 : 1);        // weight boxes per stage
+    static constexpr int KSTAGE = K2 ? 2 * kBKT : kBKT;     // reduction elements per stage
+    static constexpr int KP = kConvWarps / 4 / NB;          // converter warps per (quadrant, box)
     static constexpr int CH = (kBKT / 16) / KP;             // 16-byte chunks per converter thread and stage
-    static constexpr int STG = NA * kBM * kBKT;             // int8 staging bytes per stage
-    static constexpr int BBYTES = BN * kBKT * 2;            // bf16 activation bytes per stage
+    static constexpr int STG = NB * kBM * kBKT;             // int8 staging bytes per stage
+    static constexpr int BBYTES = BN * KSTAGE * 2;          // bf16 activation bytes per stage
     static constexpr int NDB = (UP && BN == 128) ? 1 : 2;   // accumulator buffers in TMEM
     static constexpr int ACC = NA * BN;                     // TMEM columns of one accumulator buffer
-    static constexpr int A_COLS = NA * kBKT / 2;            // TMEM columns of one A stage
+    static constexpr int A_COLS = NB * kBKT / 2;            // TMEM columns of one A stage
     static constexpr int S2 = cmin(4, (512 - NDB * ACC) / A_COLS);   // A (TMEM) + B (smem) ring
     static constexpr int S1 = cmin(12, (kSmemBudget - S2 * BBYTES) / STG);   // int8 staging ring
     static constexpr int A_BASE = NDB * ACC;                // first TMEM column of the A ring
@@ -156,8 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!w.wait(stg_empty(st), ph ^ 1u, 1)) goto a_done;
                     mbar_arrive_expect_tx(stg_full(st), C::STG);
                     const uint32_t dst = sbase + C::OFF_STG + st * C::STG;
-                    tma_load_2d(dst, &tmA0, stg_full(st), (kb + ks) * kBKT, y, pol);
-                    if (UP) tma_load_2d(dst + kBM * kBKT, &tmA1, stg_full(st), (kb + ks) * kBKT, y, pol);
+#pragma unroll
+                    for (int bx = 0; bx < C::NB; ++bx)
+                        tma_load_2d(dst + bx * kBM * kBKT, (UP && bx == 1) ? &tmA1 : &tmA0, stg_full(st),
+                                    (kb + ks) * C::KSTAGE + (UP ? 0 : bx * kBKT), y, pol);
                     issued |= 1u << st;
                     par = (par & ~(1u << st)) | (ph << st);
                     if (++st == C::S1) { st = 0; ph ^= 1u; }
@@ -182,9 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!w.wait(op_empty(st), ph ^ 1u, 2)) goto b_done;
                     mbar_arrive_expect_tx(b_full(st), C::BBYTES);
                     const uint32_t dst = sbase + C::OFF_B + st * C::BBYTES;
-                    const int x = (kb + ks) * kBKT;
-                    tma_load_2d(dst, &tmB, b_full(st), x, row, pol);
-                    tma_load_2d(dst + BN * 128, &tmB, b_full(st), x + 64, row, pol);
+                    const int x = (kb + ks) * C::KSTAGE;
+#pragma unroll
+                    for (int j = 0; j < C::KSTAGE / 64; ++j)   // 64-element (128-byte) wide boxes
+                        tma_load_2d(dst + j * BN * 128, &tmB, b_full(st), x + 64 * j, row, pol);
                     issued |= 1u << st;
                     par = (par & ~(1u << st)) | (ph << st);
                     if (++st == C::S2) { st = 0; ph ^= 1u; }
@@ -214,12 +224,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t acol = tmem_base + C::A_BASE + st * C::A_COLS;
                     const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
 #pragma unroll
-                    for (int kk = 0; kk < kBKT / 16; ++kk) {
-                        const uint64_t bdesc = desc_sw128(bbase + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
+                    for (int bx = 0; bx < C::NB; ++bx) {
 #pragma unroll
-                        for (int mat = 0; mat < C::NA; ++mat)
-                            umma_bf16_ts(dcol + mat * BN, acol + mat * (kBKT / 2) + kk * 8, bdesc, idesc,
-                                         (ks | kk) != 0);
+                        for (int kk = 0; kk < kBKT / 16; ++kk) {
+                            // K slice of the stage's activation tile; both matrices of the
+                            // up-projection use the same slices, the k-boxes of the down-projection
+                            // consecutive ones
+                            const int kg = (UP ? 0 : bx * (kBKT / 16)) + kk;
+                            const uint64_t bdesc =
+                                desc_sw128(bbase + (kg >> 2) * (BN * 128) + (kg & 3) * 32, 16, 1024);
+                            const uint32_t acc = UP ? ((ks | kk) != 0) : ((ks | bx | kk) != 0);
+                            umma_bf16_ts(dcol + (UP ? bx : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc, idesc, acc);
+                        }
                     }
                     umma_commit(op_empty(st));
                     if (++st == C::S2) { st = 0; ph ^= 1u; }
@@ -291,17 +307,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= kWarpConv0) {
         // ---- int8 staging -> bf16 A operand in TMEM ------------------------------------
         // Converter warp cw owns TMEM lane quadrant q = warp % 4 (feature rows 32q..32q+31
-        // of the tile), weight matrix `mat` and chunks [j0, j0 + CH) of the 8 16-byte
-        // chunks of each 128-byte feature row.  Lanes of one 8-lane phase read 8
+        // of the tile), weight box `box` of the stage and chunks [j0, j0 + CH) of the 8
+        // 16-byte chunks of each 128-byte feature row.  Lanes of one 8-lane phase read 8
         // different rows, whose 128-byte swizzle puts the same logical chunk in 8
         // different bank groups.
         const int cw = warp - kWarpConv0;
         const int q = warp & 3;
         const int part = cw >> 2;
-        const int mat = part / C::KP;
+        const int box = part / C::KP;
         const int j0 = (part % C::KP) * C::CH;
         const int fr = q * 32 + lane;
-        const uint32_t src_row = mat * kBM * kBKT + fr * 128;
+        const uint32_t src_row = box * kBM * kBKT + fr * 128;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         uint32_t st = 0, ph = 0, st2 = 0, ph2 = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -314,24 +330,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint4 v[C::CH];
 #pragma unroll
                 for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
-                uint32_t words[C::CH * 8];
+                const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + box * (kBKT / 2) + j0 * 8;
+                __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
+                // each 16-byte chunk (16 reduction elements = 8 TMEM columns) is stored as soon
+                // as it is converted, so the TMEM writes spread over the conversion work
 #pragma unroll
                 for (int c = 0; c < C::CH; ++c) {
-                    words[c * 8 + 0] = i8x2_to_bf16x2(v[c].x, 0x4140);
-                    words[c * 8 + 1] = i8x2_to_bf16x2(v[c].x, 0x4342);
-                    words[c * 8 + 2] = i8x2_to_bf16x2(v[c].y, 0x4140);
-                    words[c * 8 + 3] = i8x2_to_bf16x2(v[c].y, 0x4342);
-                    words[c * 8 + 4] = i8x2_to_bf16x2(v[c].z, 0x4140);
-                    words[c * 8 + 5] = i8x2_to_bf16x2(v[c].z, 0x4342);
-                    words[c * 8 + 6] = i8x2_to_bf16x2(v[c].w, 0x4140);
-                    words[c * 8 + 7] = i8x2_to_bf16x2(v[c].w, 0x4342);
+                    uint32_t words[8];
+                    words[0] = i8x2_to_bf16x2(v[c].x, 0x4140);
+                    words[1] = i8x2_to_bf16x2(v[c].x, 0x4342);
+                    words[2] = i8x2_to_bf16x2(v[c].y, 0x4140);
+                    words[3] = i8x2_to_bf16x2(v[c].y, 0x4342);
+                    words[4] = i8x2_to_bf16x2(v[c].z, 0x4140);
+                    words[5] = i8x2_to_bf16x2(v[c].z, 0x4342);
+                    words[6] = i8x2_to_bf16x2(v[c].w, 0x4140);
+                    words[7] = i8x2_to_bf16x2(v[c].w, 0x4342);
+                    tmem_st8(taddr + c * 8, words);
                 }
-                const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + mat * (kBKT / 2) + j0 * 8;
-                __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
-                if constexpr (C::CH * 8 == 32)
-                    tmem_st32(taddr, words);
-                else
-                    tmem_st16(taddr, words);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -375,7 +390,7 @@ cudaError_t launch_one_ts(const CUtensorMap &a0, const CUtensorMap &a1, const CU
 
 }  // namespace
 
-int gemm_ts_kstep() { return kBKT; }
+int gemm_ts_kstage(bool up, int bn) { return (!up && bn <= 64) ? 2 * kBKT : kBKT; }
 
 cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
                               const GemmArgs &a, int grid, cudaStream_t s)

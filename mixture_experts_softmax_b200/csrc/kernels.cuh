@@ -97,7 +97,8 @@ cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &wl, const CUtensorMap &
                               const GemmArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,
                                 int grid, cudaStream_t s);
-int gemm_ts_kstep();   // reduction elements per pipeline stage of the TMEM-operand GEMMs
+// reduction elements per pipeline stage of the TMEM-operand GEMM (up- or down-projection, tile width bn)
+int gemm_ts_kstage(bool up, int bn);
 // out[e, m, k] = in[e, k, m] for E int8 [K, M] matrices (K, M multiples of 64)
 cudaError_t launch_transpose_i8(const int8_t *in, int8_t *out, int E, int K, int M, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);

@@ -84,14 +84,18 @@ int plan_bn(int T)
 
 int bn_slot(int bn) { return bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3; }
 
-int kstep_of(const moe_ctx *h) { return h->layout == MOE_LAYOUT_PACKED ? gemm_ts_kstep() : kBK; }
+// reduction elements per pipeline stage of the up- / down-projection kernel of the handle's layout
+int kstage_of(const moe_ctx *h, bool up, int bn)
+{
+    return h->layout == MOE_LAYOUT_PACKED ? gemm_ts_kstage(up, bn) : kBK;
+}
 
 int plan_splits(const moe_ctx *h, int T, int bn)
 {
     const int per_expert = (2 * T + h->E - 1) / h->E;
     const long nt = per_expert <= bn ? 1 : (per_expert + bn - 1) / bn;
     const long tiles = static_cast<long>(h->E) * (h->d / kBM) * nt;
-    const int ksteps = h->F / kstep_of(h);
+    const int ksteps = h->F / kstage_of(h, false, bn);
     const int sms = h->num_sms > 0 ? h->num_sms : 148;
     int s = 1;
     while (s < kMaxSplits && tiles * s < 16L * sms && ksteps % (2 * s) == 0) s *= 2;
@@ -248,7 +252,7 @@ int weight_map(moe_ctx *h, const void *ptr, int kind, const CUtensorMap **out)
     int rc;
     if (h->layout == MOE_LAYOUT_PACKED)
         rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, in, static_cast<uint64_t>(h->E) * outf,
-                       gemm_ts_kstep(), kBM);
+                       128, kBM);
     else
         rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, outf, static_cast<uint64_t>(h->E) * in,
                        kBM, kBK);
@@ -367,7 +371,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.E = h->E;
     up.M = h->F;
     up.K = h->d;
-    up.ksteps = h->d / kstep_of(h);
+    up.ksteps = h->d / kstage_of(h, true, bn);
     up.splits = 1;
     up.poff = poff;
     up.rperm = rperm;
@@ -387,7 +391,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     dn.M = h->d;
     dn.K = h->F;
     dn.splits = splits;
-    dn.ksteps = h->F / kstep_of(h) / splits;
+    dn.ksteps = h->F / kstage_of(h, false, bn) / splits;
     dn.s0 = static_cast<const __nv_bfloat16 *>(s_1);
     dn.s1 = nullptr;
     dn.h = nullptr;

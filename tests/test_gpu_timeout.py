@@ -10,13 +10,17 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 
-def test_timeout_is_reported_and_context_survives():
+@pytest.mark.parametrize("layout", [0, 1], ids=["in_out", "packed"])
+def test_timeout_is_reported_and_context_survives(layout):
     import mixture_experts_softmax_b200 as m
     inp = moe_synth.make_inputs("tiny", device="cpu", T=256)
     layer = parity.to_dev(inp.layers[0])
     x = inp.x.cuda()
     rc, h = m.moe_create(256, 512, 8, 2)
     assert rc == 0
+    m.check(m.moe_set_weight_layout(h, layout))
+    if layout == m.MOE_LAYOUT_PACKED:
+        layer = m.pack_layer(h, layer)
     try:
         ref = torch.empty_like(x)
         m.check(m.moe_forward(h, 256, x, *m.layer_args(layer), ref))
