@@ -63,16 +63,6 @@ struct Waiter {
     __device__ __forceinline__ bool wait(uint32_t bar, uint32_t par, int site) const
     {
         if (mbar_try_wait(bar, par)) return true;
-#ifdef MOE_PIPE_STATS
-        const long long c0 = clock64();
-        const bool ok = wait_slow(bar, par, site);
-        atomicAdd(&g_pipe_stats[stat_base + site], static_cast<unsigned long long>(clock64() - c0));
-        return ok;
-    }
-
-    __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t par, int site) const
-    {
-#endif
         const uint64_t t0 = global_timer_ns();
         while (true) {
             if (mbar_try_wait(bar, par)) return true;
@@ -85,6 +75,20 @@ struct Waiter {
         }
     }
 };
+
+// Instrumented builds (-DMOE_PIPE_STATS): cycle counters kept per thread in registers and
+// added to g_pipe_stats once per warp at the end of the kernel.
+#ifdef MOE_PIPE_STATS
+#define PS_VAR(v) long long v = 0
+#define PS_NOW(t) const long long t = clock64()
+#define PS_ADD(v, t0) (v) += clock64() - (t0)
+#define PS_FLUSH(slot, v) atomicAdd(&g_pipe_stats[slot], static_cast<unsigned long long>(v))
+#else
+#define PS_VAR(v)
+#define PS_NOW(t)
+#define PS_ADD(v, t0)
+#define PS_FLUSH(slot, v)
+#endif
 
 // wait used only while draining after an abort: fixed 1 s limit, ignores the abort flag
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t par)

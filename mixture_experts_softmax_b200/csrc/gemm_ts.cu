@@ -144,23 +144,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     const int total = prefix[a.E];
-#ifdef MOE_PIPE_STATS
-    if (threadIdx.x == 0) atomicAdd(&g_pipe_stats[UP ? 60 : 61], static_cast<unsigned long long>(clock64()));
-#endif
-    const Waiter w{abort_flag, a.err, a.timeout_ns, UP ? 20 : 40};
+    const int SB = UP ? 0 : 32;   // first stats slot of this kernel (instrumented builds)
+    PS_NOW(t_start);
+    const Waiter w{abort_flag, a.err, a.timeout_ns, SB};
 
     if (warp == kWarpTmaA) {
         // ---- int8 weight tiles [128 f x 128 k] -> staging ring ------------------------
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();
             uint32_t st = 0, ph = 0, issued = 0, par = 0;
+            PS_VAR(c_wait);
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
                 int e, m, n, s;
                 decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
                 const int kb = s * a.ksteps;
                 const int y = e * a.M + m * kBM;
                 for (int ks = 0; ks < a.ksteps; ++ks) {
+                    PS_NOW(t0);
                     if (!w.wait(stg_empty(st), ph ^ 1u, 1)) goto a_done;
+                    PS_ADD(c_wait, t0);
                     mbar_arrive_expect_tx(stg_full(st), C::STG);
                     const uint32_t dst = sbase + C::OFF_STG + st * C::STG;
 #pragma unroll
@@ -175,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         a_done:
             for (int s = 0; s < C::S1; ++s)   // every copy issued has landed before the CTA may exit
                 if (issued & (1u << s)) wait_drain(stg_full(s), (par >> s) & 1u);
+            PS_FLUSH(SB + 1, c_wait);
         }
         __syncwarp();
     } else if (warp == kWarpTmaB) {
@@ -182,13 +185,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_last();
             uint32_t st = 0, ph = 0, issued = 0, par = 0;
+            PS_VAR(c_bwait);
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
                 int e, m, n, s;
                 decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
                 const int kb = s * a.ksteps;
                 const int row = poff[e] + n * BN;
                 for (int ks = 0; ks < a.ksteps; ++ks) {
+                    PS_NOW(t0);
                     if (!w.wait(op_empty(st), ph ^ 1u, 2)) goto b_done;
+                    PS_ADD(c_bwait, t0);
                     mbar_arrive_expect_tx(b_full(st), C::BBYTES);
                     const uint32_t dst = sbase + C::OFF_B + st * C::BBYTES;
                     const int x = (kb + ks) * C::KSTAGE;
@@ -203,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         b_done:
             for (int s = 0; s < C::S2; ++s)
                 if (issued & (1u << s)) wait_drain(b_full(s), (par >> s) & 1u);
+            PS_FLUSH(SB + 2, c_bwait);
         }
         __syncwarp();
     } else if (warp == kWarpMma) {
@@ -211,15 +218,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = idesc_ts<BN>();
             uint32_t st = 0, ph = 0;
             int it = 0;
+            PS_VAR(c_acc);
+            PS_VAR(c_a);
+            PS_VAR(c_b);
+            PS_VAR(c_issue);
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
                 const int b = it % C::NDB;
                 const uint32_t aph = (it / C::NDB) & 1;
+                PS_NOW(t0);
                 if (!w.wait(acc_empty(b), aph ^ 1u, 3)) break;
+                PS_ADD(c_acc, t0);
                 tc_fence_after();
                 const uint32_t dcol = tmem_base + b * C::ACC;
                 bool ok = true;
                 for (int ks = 0; ks < a.ksteps; ++ks) {
-                    if (!w.wait(a_full(st), ph, 4) || !w.wait(b_full(st), ph, 5)) { ok = false; break; }
+                    PS_NOW(t1);
+                    if (!w.wait(a_full(st), ph, 4)) { ok = false; break; }
+                    PS_ADD(c_a, t1);
+                    PS_NOW(t2);
+                    if (!w.wait(b_full(st), ph, 5)) { ok = false; break; }
+                    PS_ADD(c_b, t2);
+                    PS_NOW(t3);
                     tc_fence_after();
                     const uint32_t acol = tmem_base + C::A_BASE + st * C::A_COLS;
                     const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
@@ -238,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     umma_commit(op_empty(st));
+                    PS_ADD(c_issue, t3);
                     if (++st == C::S2) { st = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
@@ -245,19 +265,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             umma_commit(drain_bar);          // all MMAs issued above have completed after this
             wait_drain(drain_bar, 0);
+            PS_FLUSH(SB + 3, c_acc);
+            PS_FLUSH(SB + 4, c_a);
+            PS_FLUSH(SB + 5, c_b);
+            PS_FLUSH(SB + 6, c_issue);
         }
         __syncwarp();
     } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
         // ---- epilogue: TMEM -> registers -> global -----------------------------------
         const int ew = warp - kWarpEpi0;
         int it = 0;
+        PS_VAR(c_ewait);
+        PS_VAR(c_ework);
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             int e, m, n, s;
             decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
             const int b = it % C::NDB;
             const uint32_t aph = (it / C::NDB) & 1;
+            PS_NOW(t0);
             const bool ok = __all_sync(0xffffffffu, w.wait(acc_full(b), aph, 6));
             if (!ok) break;
+            PS_ADD(c_ewait, t0);
+            PS_NOW(t1);
             tc_fence_after();
             const int f = m * kBM + ew * 32 + lane;
             const uint32_t tl = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * C::ACC;
@@ -303,6 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty(b));
+            PS_ADD(c_ework, t1);
+        }
+        if (lane == 0) {
+            PS_FLUSH(SB + 7, c_ewait);
+            PS_FLUSH(SB + 8, c_ework);
         }
     } else if (warp >= kWarpConv0) {
         // ---- int8 staging -> bf16 A operand in TMEM ------------------------------------
@@ -320,11 +354,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t src_row = box * kBM * kBKT + fr * 128;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         uint32_t st = 0, ph = 0, st2 = 0, ph2 = 0;
+        PS_VAR(c_cwait);
+        PS_VAR(c_cwork);
+        PS_VAR(c_cst);
+        PS_VAR(c_ctail);
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             bool ok = true;
             for (int ks = 0; ks < a.ksteps; ++ks) {
+                PS_NOW(t0);
                 ok = __all_sync(0xffffffffu, w.wait(stg_full(st), ph, 7) && w.wait(op_empty(st2), ph2 ^ 1u, 8));
                 if (!ok) break;
+                PS_ADD(c_cwait, t0);
+                PS_NOW(t1);
                 tc_fence_after();
                 const uint32_t src = sbase + C::OFF_STG + st * C::STG + src_row;
                 uint4 v[C::CH];
@@ -347,17 +388,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     words[7] = i8x2_to_bf16x2(v[c].w, 0x4342);
                     tmem_st8(taddr + c * 8, words);
                 }
+                PS_ADD(c_cwork, t1);
+                PS_NOW(t2);
                 tmem_wait_st();
+                PS_ADD(c_cst, t2);
+                PS_NOW(t3);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(stg_empty(st));
                     mbar_arrive(a_full(st2));
                 }
+                PS_ADD(c_ctail, t3);
                 if (++st == C::S1) { st = 0; ph ^= 1u; }
                 if (++st2 == C::S2) { st2 = 0; ph2 ^= 1u; }
             }
             if (!ok) break;
+        }
+        if (lane == 0) {
+            PS_FLUSH(SB + 9, c_cwait);
+            PS_FLUSH(SB + 10, c_cwork);
+            PS_FLUSH(SB + 11, c_cst);
+            PS_FLUSH(SB + 12, c_ctail);
         }
     }
 
@@ -368,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 #ifdef MOE_PIPE_STATS
-    if (threadIdx.x == 0) atomicAdd(&g_pipe_stats[UP ? 62 : 63], static_cast<unsigned long long>(clock64()));
+    if (threadIdx.x == 0) PS_FLUSH(SB + 0, clock64() - t_start);
 #endif
 }
 
