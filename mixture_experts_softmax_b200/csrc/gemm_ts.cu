@@ -17,7 +17,9 @@
 //     with tcgen05.st (one 32-bit TMEM column holds two consecutive k);
 //   - a second TMA producer copies the bf16 activation tile [BN r x 128 k] into the
 //     shared-memory operand ring;
-//   - one thread issues tcgen05.mma with A from TMEM and B from shared memory;
+//   - one thread issues tcgen05.mma with A from TMEM and B from shared memory; where a
+//     stage holds two weight boxes with accumulators of their own, two threads on different
+//     SM sub-partitions (warps 1 and 3) issue one box each;
 //   - 4 epilogue warps apply the same fused epilogues as the shared-memory variant.
 // Shared-memory traffic per weight byte is the TMA write plus one read (against
 // also a bf16 write and an MMA read of 2 bytes each when the dequantised tile goes
@@ -29,7 +31,7 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 768;                  // 24 warps
-constexpr int kWarpTmaA = 0, kWarpMma = 1, kWarpTmaB = 2;
+constexpr int kWarpTmaA = 0, kWarpMma = 1, kWarpTmaB = 2, kWarpMma2 = 3;
 constexpr int kWarpEpi0 = 4;                   // warps 4..7: epilogue (TMEM lanes 0..127)
 constexpr int kWarpConv0 = 8;                  // warps 8..23: converters
 constexpr int kConvWarps = 16;
@@ -43,7 +45,7 @@ static_assert(kWarpConv0 % 4 == 0, "converter warp w must own TMEM lane quadrant
 // moves 32 KB), the down-projection with 128-route tiles one box.
 template <bool UP, int BN>
 struct CfgTS {
-    static constexpr int NA = UP ? 2 : 1;                   // weight matrices = accumulators
+    static constexpr int NA = UP ? 2 : 1;                   // weight matrices
     static constexpr bool K2 = !UP && BN <= 64;             // two k-boxes per stage
     static constexpr int NB = UP ? 2 : (K2 ? 2 : 1);        // weight boxes per stage
     static constexpr int KSTAGE = K2 ? 2 * kBKT : kBKT;     // reduction elements per stage
@@ -52,7 +54,14 @@ struct CfgTS {
     static constexpr int STG = NB * kBM * kBKT;             // int8 staging bytes per stage
     static constexpr int BBYTES = BN * KSTAGE * 2;          // bf16 activation bytes per stage
     static constexpr int NDB = (UP && BN == 128) ? 1 : 2;   // accumulator buffers in TMEM
-    static constexpr int ACC = NA * BN;                     // TMEM columns of one accumulator buffer
+    // Two MMA issuers, one per box of a stage, each into an accumulator of its own: the
+    // up-projection (one accumulator per matrix anyway) and the narrow down-projection (one per
+    // k-box, summed by the epilogue).  The converter warps keep every SM sub-partition's issue
+    // slots busy, and a single issuing thread, which spends several instructions per MMA, then
+    // falls behind the tensor core at the small N of decode-sized tiles.
+    static constexpr bool DUAL = UP || (K2 && BN <= 32);
+    static constexpr int NACC = DUAL ? 2 : 1;               // accumulators per tile
+    static constexpr int ACC = NACC * BN;                   // TMEM columns of one accumulator buffer
     static constexpr int A_COLS = NB * kBKT / 2;            // TMEM columns of one A stage
     static constexpr int S2 = cmin(4, (512 - NDB * ACC) / A_COLS);   // A (TMEM) + B (smem) ring
     static constexpr int S1 = cmin(12, (kSmemBudget - S2 * BBYTES) / STG);   // int8 staging ring
@@ -61,8 +70,8 @@ struct CfgTS {
     static constexpr int OFF_STG = 0;
     static constexpr int OFF_B = OFF_STG + S1 * STG;
     static constexpr int OFF_BAR = OFF_B + S2 * BBYTES;
-    // barriers: stg_full[S1] stg_empty[S1] a_full[S2] b_full[S2] op_empty[S2] acc_full[NDB] acc_empty[NDB] drain
-    static constexpr int NBAR = 2 * S1 + 3 * S2 + 2 * NDB + 1;
+    // barriers: stg_full[S1] stg_empty[S1] a_full[S2] b_full[S2] op_empty[S2] acc_full[NDB] acc_empty[NDB] drain[2]
+    static constexpr int NBAR = 2 * S1 + 3 * S2 + 2 * NDB + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int MISC_BYTES = 16 + 2 * 4 * 40;
     static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;
@@ -116,13 +125,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < C::S2; ++s) {
             mbar_init(a_full(s), kConvWarps);
             mbar_init(b_full(s), 1);
-            mbar_init(op_empty(s), 1);
+            mbar_init(op_empty(s), C::NACC);   // one commit per issuer
         }
         for (int b = 0; b < C::NDB; ++b) {
-            mbar_init(acc_full(b), 1);
+            mbar_init(acc_full(b), C::NACC);
             mbar_init(acc_empty(b), 4);
         }
         mbar_init(drain_bar, 1);
+        mbar_init(drain_bar + 8, 1);
         *abort_flag = 0u;
         prefix[0] = 0;
         for (int e = 0; e <= a.E; ++e) poff[e] = a.poff[e];
@@ -212,8 +222,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             PS_FLUSH(SB + 2, c_bwait);
         }
         __syncwarp();
-    } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMma || (C::DUAL && warp == kWarpMma2)) {
         // ---- tensor-core issue: A from TMEM, B from shared memory --------------------
+        // with two issuers, issuer i takes box i of every stage into accumulator i
+        const int mine = warp == kWarpMma ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_ts<BN>();
             uint32_t st = 0, ph = 0;
@@ -244,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
 #pragma unroll
                     for (int bx = 0; bx < C::NB; ++bx) {
+                        if (C::DUAL && bx != mine) continue;
 #pragma unroll
                         for (int kk = 0; kk < kBKT / 16; ++kk) {
                             // K slice of the stage's activation tile; both matrices of the
@@ -252,8 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int kg = (UP ? 0 : bx * (kBKT / 16)) + kk;
                             const uint64_t bdesc =
                                 desc_sw128(bbase + (kg >> 2) * (BN * 128) + (kg & 3) * 32, 16, 1024);
-                            const uint32_t acc = UP ? ((ks | kk) != 0) : ((ks | bx | kk) != 0);
-                            umma_bf16_ts(dcol + (UP ? bx : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc, idesc, acc);
+                            const uint32_t acc = C::DUAL ? ((ks | kk) != 0) : ((ks | bx | kk) != 0);
+                            umma_bf16_ts(dcol + (C::DUAL ? bx : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc,
+                                         idesc, acc);
                         }
                     }
                     umma_commit(op_empty(st));
@@ -263,8 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 umma_commit(acc_full(b));
             }
-            umma_commit(drain_bar);          // all MMAs issued above have completed after this
-            wait_drain(drain_bar, 0);
+            umma_commit(drain_bar + 8 * mine);   // all MMAs this thread issued have completed after this
+            wait_drain(drain_bar + 8 * mine, 0);
             PS_FLUSH(SB + 3, c_acc);
             PS_FLUSH(SB + 4, c_a);
             PS_FLUSH(SB + 5, c_b);
@@ -316,7 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float v[16];
                     __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
                     tmem_ld16(tl + c, v);
-                    tmem_wait_ld();
+                    if constexpr (C::DUAL) {   // the two k-box accumulators, summed in this order
+                        float v1[16];
+                        tmem_ld16(tl + BN + c, v1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] += v1[i];
+                    } else {
+                        tmem_wait_ld();
+                    }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int route = __ldg(a.rperm + row0 + c + i);
