@@ -30,14 +30,16 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 768;                  // 24 warps
+constexpr int kThreads = 640;                  // 20 warps
 constexpr int kWarpTmaA = 0, kWarpMma = 1, kWarpTmaB = 2, kWarpMma2 = 3;
-constexpr int kWarpEpi0 = 4;                   // warps 4..7: epilogue (TMEM lanes 0..127)
-constexpr int kWarpConv0 = 8;                  // warps 8..23: converters
-constexpr int kConvWarps = 16;
+constexpr int kWarpEpi0 = 4;                   // warps 4..11: epilogue, two per TMEM lane quadrant
+constexpr int kEpiWarps = 8;
+constexpr int kWarpConv0 = 12;                 // warps 12..19: converters, two per TMEM lane quadrant
+constexpr int kConvWarps = 8;
 constexpr int kBKT = 128;                      // reduction elements per stage
 constexpr int kSmemBudget = 208 * 1024;
-static_assert(kWarpConv0 % 4 == 0, "converter warp w must own TMEM lane quadrant w % 4");
+static_assert(kWarpConv0 % 4 == 0 && kWarpEpi0 % 4 == 0, "warp w must own TMEM lane quadrant w % 4");
+static_assert(kWarpConv0 + kConvWarps == kThreads / 32 && kWarpEpi0 + kEpiWarps == kWarpConv0, "warp roles");
 
 // Weight tiles are [128 features x 128 reduction elements] int8 "boxes" of 16 KB.  A pipeline
 // stage carries NB boxes: the up-projection one box of each of its two matrices (same k), the
@@ -78,7 +80,7 @@ struct CfgTS {
     static_assert(S1 >= 2 && S2 >= 2, "rings too shallow");
     static_assert(SMEM <= 227 * 1024, "shared memory over the per-CTA limit");
     static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
-    static_assert(CH * 8 == 16 || CH * 8 == 32, "a converter thread stores 16 or 32 TMEM columns");
+    static_assert(KP >= 1 && CH * KP == kBKT / 16, "converter warps must split the 8 chunks of a row");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is 16..256 in steps of 16");
 };
 
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < C::NDB; ++b) {
             mbar_init(acc_full(b), C::NACC);
-            mbar_init(acc_empty(b), 4);
+            mbar_init(acc_empty(b), kEpiWarps);
         }
         mbar_init(drain_bar, 1);
         mbar_init(drain_bar + 8, 1);
@@ -285,9 +287,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             PS_FLUSH(SB + 6, c_issue);
         }
         __syncwarp();
-    } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
+    } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + kEpiWarps) {
         // ---- epilogue: TMEM -> registers -> global -----------------------------------
-        const int ew = warp - kWarpEpi0;
+        // warp (q, hc): TMEM lane quadrant q = warp % 4, column half hc of the tile (narrowest
+        // tiles: the first four warps take all 16 columns, the others only hand the buffer back)
+        const int q = warp & 3;
+        const int hc = (warp - kWarpEpi0) >> 2;
+        constexpr int kCols = BN >= 32 ? BN / 2 : BN;
+        const int c0 = BN >= 32 ? hc * kCols : 0;
+        const int c1 = BN >= 32 || hc == 0 ? c0 + kCols : c0;
         int it = 0;
         PS_VAR(c_ewait);
         PS_VAR(c_ework);
@@ -302,14 +310,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             PS_ADD(c_ewait, t0);
             PS_NOW(t1);
             tc_fence_after();
-            const int f = m * kBM + ew * 32 + lane;
-            const uint32_t tl = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * C::ACC;
+            const int f = m * kBM + q * 32 + lane;
+            const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::ACC;
             const int row0 = poff[e] + n * BN;
             if constexpr (UP) {
                 const float sa = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
                 const float sb = __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
+                for (int c = c0; c < c1; c += 16) {
                     float va[16], vb[16];
                     __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
                     tmem_ld16(tl + c, va);
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 const float sc = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
+                for (int c = c0; c < c1; c += 16) {
                     float v[16];
                     __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
                     tmem_ld16(tl + c, v);
