@@ -31,7 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/sec at Grok-1 shape; % of HBM / bf16 tensor-pipe roofline"
-KERNELS = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm")
+KERNELS = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm", "route_small")
 
 
 def parse():

@@ -176,8 +176,10 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns);
  * moe_set_profiling(h, 1) starts recording around each kernel of every forward;
  * moe_get_kernel_times synchronises on those events and returns, per kernel id
  * (0 router, 1 dispatch, 2 gather, 3 up-projection, 4 down-projection,
- * 5 combine, 6 pre-norm), the total milliseconds and the launch count since the
- * previous call, then resets them.  n = capacity of ms/launches (7 suffices).
+ * 5 combine, 6 pre-norm, 7 small-batch routing: router, dispatch and gather in
+ * one launch, used instead of 0-2 when T <= 32), the total milliseconds and the
+ * launch count since the previous call, then resets them.  n = capacity of
+ * ms/launches (8 suffices).
  */
 MOE_API int moe_set_profiling(moe_handle h, int on);
 MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);

@@ -31,7 +31,7 @@ MOE_LAYOUT_IN_OUT = 0
 MOE_LAYOUT_PACKED = 1
 MOE_NOALLOC_MAX_TOKENS = 65536
 
-KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm")
+KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm", "route_small")
 
 # every symbol include/moe.h declares
 EXPORTS = (

@@ -47,7 +47,6 @@ static_assert(kWarpConv0 + kConvWarps == kThreads / 32 && kWarpEpi0 + kEpiWarps 
 // moves 32 KB), the down-projection with 128-route tiles one box.
 template <bool UP, int BN>
 struct CfgTS {
-    static constexpr int NA = UP ? 2 : 1;                   // weight matrices
     static constexpr bool K2 = !UP && BN <= 64;             // two k-boxes per stage
     static constexpr int NB = UP ? 2 : (K2 ? 2 : 1);        // weight boxes per stage
     static constexpr int KSTAGE = K2 ? 2 * kBKT : kBKT;     // reduction elements per stage

@@ -38,11 +38,9 @@ struct DispatchArgs {
 };
 
 struct GatherArgs {
-    int d, max_rows;
-    const int *poff_end;        // &poff[E]: number of padded rows (device)
-    const int *rperm;
+    int d;
     const __nv_bfloat16 *x;     // [T, d]
-    __nv_bfloat16 *xp;          // [rows, d]
+    __nv_bfloat16 *xp;          // [rows, d]; only the rows of real routes are written
 };
 
 // one grouped GEMM of the layer:  for every expert e and padded row r of e
@@ -87,7 +85,13 @@ struct NormArgs {
 
 cudaError_t launch_router(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
-cudaError_t launch_gather(const GatherArgs &a, cudaStream_t s);
+// Xp[slot_of_route[r]] = x[r / 2] for the 2T routes
+cudaError_t launch_gather(const GatherArgs &a, int T, const int *slot_of_route, cudaStream_t s);
+// router + dispatch + gather in one launch for T <= route_small_max_tokens(); `ticket` is a
+// zero-initialised device word owned by the caller (left at 0 after the launch)
+int route_small_max_tokens();
+cudaError_t launch_route_small(const RouteArgs &ra, const DispatchArgs &da, const GatherArgs &ga, unsigned int *ticket,
+                               cudaStream_t s);
 cudaError_t launch_gemm_up(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
                            const GemmArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_gemm_down(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,

@@ -14,7 +14,7 @@ using namespace moe;
 
 namespace {
 
-enum KernelId { K_ROUTER = 0, K_DISPATCH, K_GATHER, K_UP, K_DOWN, K_COMBINE, K_PRENORM };
+enum KernelId { K_ROUTER = 0, K_DISPATCH, K_GATHER, K_UP, K_DOWN, K_COMBINE, K_PRENORM, K_ROUTE_SMALL };
 
 struct DevBuf {
     void *ptr = nullptr;
@@ -49,7 +49,7 @@ struct moe_ctx {
     DevBuf b_h;        // bf16 [rows, F]
     DevBuf b_slots;    // fp32 [splits, T, 2, d]
     DevBuf b_stage;    // bf16 [T, d] x2: host-API input/output staging, block pre-norm output
-    int *err = nullptr;
+    int *err = nullptr;     // 256 zeroed bytes: word 0 the device error word, word 32 the routing ticket
     int rows_cap = 0;       // rows the xp / h buffers hold
     int route_cap = 0;      // T the route buffer holds
     int map_gen = 0;        // bumps when b_xp / b_h move
@@ -347,7 +347,6 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     float *gate = reinterpret_cast<float *>(rw + L.gate);
     int *poff = rw + L.poff;
     int *rperm = static_cast<int *>(h->b_rperm.ptr);
-    const int rows = rows_for(h, T, bn);
 
     const bool ts = h->layout == MOE_LAYOUT_PACKED;
     const CUtensorMap *m_wl, *m_wv, *m_w1, *m_xp, *m_h;
@@ -357,14 +356,18 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     if ((rc = act_maps(h, bn, &m_xp, &m_h)) != MOE_OK) return rc;
 
     RouteArgs ra{T, h->d, static_cast<const __nv_bfloat16 *>(x), router_w, h->bias, idx, gate};
-    if (timed(h, K_ROUTER, s, [&] { return launch_router(ra, s); }) != cudaSuccess) return MOE_ECUDA;
-
     DispatchArgs da{T, h->E, bn, idx, rw + L.counts, rw + L.offsets, poff, rw + L.perm, rperm, rw + L.slot};
-    if (timed(h, K_DISPATCH, s, [&] { return launch_dispatch(da, s); }) != cudaSuccess) return MOE_ECUDA;
-
-    GatherArgs ga{h->d, rows, poff + h->E, rperm, static_cast<const __nv_bfloat16 *>(x),
-                  static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
-    if (timed(h, K_GATHER, s, [&] { return launch_gather(ga, s); }) != cudaSuccess) return MOE_ECUDA;
+    GatherArgs ga{h->d, static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
+    if (T <= route_small_max_tokens()) {
+        unsigned int *ticket = reinterpret_cast<unsigned int *>(h->err + 32);
+        if (timed(h, K_ROUTE_SMALL, s, [&] { return launch_route_small(ra, da, ga, ticket, s); }) != cudaSuccess)
+            return MOE_ECUDA;
+    } else {
+        if (timed(h, K_ROUTER, s, [&] { return launch_router(ra, s); }) != cudaSuccess) return MOE_ECUDA;
+        if (timed(h, K_DISPATCH, s, [&] { return launch_dispatch(da, s); }) != cudaSuccess) return MOE_ECUDA;
+        if (timed(h, K_GATHER, s, [&] { return launch_gather(ga, T, rw + L.slot, s); }) != cudaSuccess)
+            return MOE_ECUDA;
+    }
 
     GemmArgs up{};
     up.T = T;

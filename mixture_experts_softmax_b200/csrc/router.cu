@@ -3,99 +3,18 @@
 // RMSNorm of the residual block ("Transformer stack and language model head").
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "route_common.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kRouterWarps = 8;       // warps per block
+constexpr int kRouterWarps = kRouteTokenThreads / 32;   // warps per block
 constexpr int kTokensPerWarp = 4;     // large-T variant: tokens sharing each router-weight load
 constexpr int kSmallT = 256;          // up to this many tokens: one block per token
 
-// x (8 bf16 packed in a uint4) times 8 rows of the [d, 8] fp32 router weight starting at `row`
-__device__ __forceinline__ void dot8(const uint4 &v, const float4 *w4, int row, float (&acc)[kExperts])
-{
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float x0 = __uint_as_float(wv[q] << 16);
-        const float x1 = __uint_as_float(wv[q] & 0xffff0000u);
-        const int r = row + 2 * q;
-        const float4 a0 = __ldg(w4 + r * 2), a1 = __ldg(w4 + r * 2 + 1);
-        const float4 b0 = __ldg(w4 + r * 2 + 2), b1 = __ldg(w4 + r * 2 + 3);
-        acc[0] = fmaf(x0, a0.x, acc[0]); acc[1] = fmaf(x0, a0.y, acc[1]);
-        acc[2] = fmaf(x0, a0.z, acc[2]); acc[3] = fmaf(x0, a0.w, acc[3]);
-        acc[4] = fmaf(x0, a1.x, acc[4]); acc[5] = fmaf(x0, a1.y, acc[5]);
-        acc[6] = fmaf(x0, a1.z, acc[6]); acc[7] = fmaf(x0, a1.w, acc[7]);
-        acc[0] = fmaf(x1, b0.x, acc[0]); acc[1] = fmaf(x1, b0.y, acc[1]);
-        acc[2] = fmaf(x1, b0.z, acc[2]); acc[3] = fmaf(x1, b0.w, acc[3]);
-        acc[4] = fmaf(x1, b1.x, acc[4]); acc[5] = fmaf(x1, b1.y, acc[5]);
-        acc[6] = fmaf(x1, b1.z, acc[6]); acc[7] = fmaf(x1, b1.w, acc[7]);
-    }
-}
-
-// logits (+ bias) -> top-2 on the fp32 logits (strictly larger wins, equal logits keep
-// the lower expert index) and the fp32 softmax probabilities of the two picks
-__device__ __forceinline__ void select_top2(float (&acc)[kExperts], const float *bias, int t, int *idx, float *gate)
-{
-    if (bias) {
-#pragma unroll
-        for (int e = 0; e < kExperts; ++e) acc[e] += __ldg(bias + e);
-    }
-    int e0 = 0;
-#pragma unroll
-    for (int e = 1; e < kExperts; ++e)
-        if (acc[e] > acc[e0]) e0 = e;
-    int e1 = (e0 == 0) ? 1 : 0;
-#pragma unroll
-    for (int e = 0; e < kExperts; ++e)
-        if (e != e0 && acc[e] > acc[e1]) e1 = e;
-    const float m = acc[e0];
-    float s = 0.f;
-#pragma unroll
-    for (int e = 0; e < kExperts; ++e) s += expf(acc[e] - m);
-    const float inv = 1.f / s;
-    idx[2 * t] = e0;
-    idx[2 * t + 1] = e1;
-    gate[2 * t] = inv;                        // exp(0) / s
-    gate[2 * t + 1] = expf(acc[e1] - m) * inv;
-}
-
-// Few tokens: one block per token, the 256 threads split d; every thread issues all
-// its loads at once (one memory latency), then a fixed-order reduction (lane tree,
-// then the 8 warp partials in warp order) gives the logits.
-__global__ void __launch_bounds__(kRouterWarps * 32) router_small_kernel(RouteArgs a)
-{
-    __shared__ float part[kRouterWarps][kExperts];
-    const int t = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * a.d);
-    const float4 *w4 = reinterpret_cast<const float4 *>(a.w);
-    float acc[kExperts];
-#pragma unroll
-    for (int e = 0; e < kExperts; ++e) acc[e] = 0.f;
-    const int chunks = a.d >> 3;
-#pragma unroll 4
-    for (int c = threadIdx.x; c < chunks; c += blockDim.x) dot8(__ldg(xr + c), w4, c * 8, acc);
-#pragma unroll
-    for (int e = 0; e < kExperts; ++e) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int e = 0; e < kExperts; ++e) part[warp][e] = acc[e];
-    }
-    __syncthreads();
-    if (threadIdx.x != 0) return;
-#pragma unroll
-    for (int e = 0; e < kExperts; ++e) {
-        float v = 0.f;
-        for (int w = 0; w < kRouterWarps; ++w) v += part[w][e];
-        acc[e] = v;
-    }
-    select_top2(acc, a.bias, t, a.idx, a.gate);
-}
+// Few tokens: one block per token (route_token, shared with the fused small-batch routing).
+__global__ void __launch_bounds__(kRouteTokenThreads) router_small_kernel(RouteArgs a) { route_token(a, blockIdx.x); }
 
 // Many tokens: each warp takes 4 tokens, so every router-weight load feeds 4 tokens and
 // the 8 warps of a block share those loads through L1; lane partial sums are reduced
@@ -193,7 +112,7 @@ cudaError_t launch_router(const RouteArgs &a, cudaStream_t s)
 {
     if (a.T <= 0) return cudaSuccess;
     if (a.T <= kSmallT) {
-        router_small_kernel<<<a.T, kRouterWarps * 32, 0, s>>>(a);
+        router_small_kernel<<<a.T, kRouteTokenThreads, 0, s>>>(a);
     } else {
         const int per_block = kRouterWarps * kTokensPerWarp;
         router_kernel<<<(a.T + per_block - 1) / per_block, kRouterWarps * 32, 0, s>>>(a);

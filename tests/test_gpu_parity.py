@@ -124,6 +124,22 @@ def test_kernel_times_reported(m, tiny_inputs, tiny_handle):
         assert times[k][1] == 3 and times[k][0] > 0
 
 
+def test_small_batch_routing_is_one_launch(m, tiny_inputs, tiny_handle):
+    """T <= 32 runs router, dispatch and gather as one launch (kernel id 7)."""
+    h, layer, _ = tiny_handle
+    x = tiny_inputs.x[:8].cuda()
+    out = torch.empty_like(x)
+    m.check(m.moe_set_profiling(h, True))
+    for _ in range(3):
+        m.check(m.moe_forward(h, 8, x, *m.layer_args(layer), out))
+    rc, times = m.moe_get_kernel_times(h)
+    m.check(m.moe_set_profiling(h, False))
+    assert rc == 0
+    assert times["route_small"][1] == 3 and times["route_small"][0] > 0
+    for k in ("router", "dispatch", "gather"):
+        assert times[k][1] == 0
+
+
 def test_pack_weight_is_a_transpose(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
