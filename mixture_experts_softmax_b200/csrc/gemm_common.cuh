@@ -113,4 +113,42 @@ __device__ __forceinline__ void decode_tile(int tile, const int *prefix, const i
 }
 
 
+// The persistent CTAs' work list.  Tiles fill whole waves of gridDim.x CTAs; the r tiles of
+// a last, partial wave are each cut along the reduction into P = gridDim.x / r pieces
+// (stream-K for the last wave only), so every CTA runs the same number of whole tiles and
+// at most one piece.  A piece leaves its fp32 accumulator in a workspace; the piece that
+// finishes last (a ticket per tile) adds the P partial sums in piece order and applies the
+// tile's epilogue.  P < 2 means no pieces.
+struct WorkList {
+    int whole;    // items [0, whole): whole tiles 0 .. whole-1
+    int P;        // pieces per split tile
+    int items;    // whole + (tiles - whole) * P
+};
+
+__device__ __forceinline__ WorkList make_work_list(int tiles, int grid, int ksteps)
+{
+    WorkList q;
+    const int r = tiles % grid;
+    int P = r ? grid / r : 0;
+    if (P > ksteps) P = ksteps;
+    if (P < 2) P = 0;
+    q.P = P;
+    q.whole = P ? tiles - r : tiles;
+    q.items = q.whole + (P ? r * P : 0);
+    return q;
+}
+
+struct WorkItem {
+    int tile;     // tile index (decode_tile)
+    int k0, k1;   // stages [k0, k1) of the tile's split
+    int piece;    // -1: the whole tile; else the piece's slot in the partial-sum workspace
+};
+
+__device__ __forceinline__ WorkItem work_item(const WorkList &q, int i, int ksteps)
+{
+    if (i < q.whole) return {i, 0, ksteps, -1};
+    const int j = i - q.whole, t = j / q.P, p = j - t * q.P;
+    return {q.whole + t, p * ksteps / q.P, (p + 1) * ksteps / q.P, j};
+}
+
 }  // namespace moe

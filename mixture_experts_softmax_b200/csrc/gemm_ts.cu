@@ -91,6 +91,78 @@ __device__ __forceinline__ constexpr uint32_t idesc_ts()
            (static_cast<uint32_t>(kBM >> 4) << 24);
 }
 
+// The tile epilogue on columns c .. c+15 of one accumulator row (TMEM lane = feature f),
+// from the full-K sums x0 (and x1: the second matrix, or the second k-box):
+//   up-projection:   H[r, f] = bf16( gelu(s0 * x0) * (s1 * x1) )
+//   down-projection: slot[s, t, j, f] = gate[t, j] * s0 * (x0 + x1)   (k-box sums in this order)
+// rows r = row0 + c + i whose route id is -1 (padding) are skipped.
+struct EpiOut {
+    const int *rperm;
+    const float *gate;
+    __nv_bfloat16 *h;
+    float *slots;
+    int M, T;
+};
+
+template <bool UP, int NACC>
+__device__ __forceinline__ void epilogue_chunk(const EpiOut &a, int row0, int c, int f, int s, float sc0, float sc1,
+                                               const float (&x0)[16], const float (&x1)[16])
+{
+    if constexpr (UP) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = row0 + c + i;
+            if (__ldg(a.rperm + r) >= 0)
+                a.h[static_cast<size_t>(r) * a.M + f] = __float2bfloat16_rn(gelu_tanh(sc0 * x0[i]) * (sc1 * x1[i]));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int route = __ldg(a.rperm + row0 + c + i);
+            if (route >= 0) {
+                const float v = NACC == 2 ? x0[i] + x1[i] : x0[i];
+                const float g = __ldg(a.gate + route);
+                const size_t o =
+                    ((static_cast<size_t>(s) * a.T + (route >> 1)) * 2 + (route & 1)) * static_cast<size_t>(a.M) + f;
+                a.slots[o] = g * (sc0 * v);
+            }
+        }
+    }
+}
+
+// The last piece of a split tile: add the P pieces' partial sums of this thread's row (p0 =
+// piece 0's row, pieces kBM * ACC floats apart) in piece order, then the tile epilogue.  Out
+// of line: it runs at most once per split tile and would otherwise raise the register
+// pressure of the whole kernel.
+template <bool UP, int BN, int NACC, int ACC>
+__device__ __noinline__ void finish_pieces(const EpiOut a, const float *p0, int P, int c0, int c1, int row0, int f,
+                                           int s, float sc0, float sc1)
+{
+    const size_t pstride = static_cast<size_t>(kBM) * ACC;
+    for (int c = c0; c < c1; c += 16) {
+        float x0[16], x1[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x0[i] = x1[i] = 0.f;
+        for (int p = 0; p < P; ++p) {
+            const float4 *r0 = reinterpret_cast<const float4 *>(p0 + p * pstride + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 u = __ldcg(r0 + i);
+                x0[4 * i] += u.x; x0[4 * i + 1] += u.y; x0[4 * i + 2] += u.z; x0[4 * i + 3] += u.w;
+            }
+            if constexpr (NACC == 2) {
+                const float4 *r1 = reinterpret_cast<const float4 *>(p0 + p * pstride + BN + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 u = __ldcg(r1 + i);
+                    x1[4 * i] += u.x; x1[4 * i + 1] += u.y; x1[4 * i + 2] += u.z; x1[4 * i + 3] += u.w;
+                }
+            }
+        }
+        epilogue_chunk<UP, NACC>(a, row0, c, f, s, sc0, sc1, x0, x1);
+    }
+}
+
 template <bool UP, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_ts_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -155,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     const int total = prefix[a.E];
+    const WorkList wl = a.part ? make_work_list(total, gridDim.x, a.ksteps) : WorkList{total, 0, total};
     const int SB = UP ? 0 : 32;   // first stats slot of this kernel (instrumented builds)
     PS_NOW(t_start);
     const Waiter w{abort_flag, a.err, a.timeout_ns, SB};
@@ -165,12 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = l2_policy_evict_first();
             uint32_t st = 0, ph = 0, issued = 0, par = 0;
             PS_VAR(c_wait);
-            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            for (int item = blockIdx.x; item < wl.items && !*abort_flag; item += gridDim.x) {
+                const WorkItem wi = work_item(wl, item, a.ksteps);
                 int e, m, n, s;
-                decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
                 const int kb = s * a.ksteps;
                 const int y = e * a.M + m * kBM;
-                for (int ks = 0; ks < a.ksteps; ++ks) {
+                for (int ks = wi.k0; ks < wi.k1; ++ks) {
                     PS_NOW(t0);
                     if (!w.wait(stg_empty(st), ph ^ 1u, 1)) goto a_done;
                     PS_ADD(c_wait, t0);
@@ -197,12 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = l2_policy_evict_last();
             uint32_t st = 0, ph = 0, issued = 0, par = 0;
             PS_VAR(c_bwait);
-            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            for (int item = blockIdx.x; item < wl.items && !*abort_flag; item += gridDim.x) {
+                const WorkItem wi = work_item(wl, item, a.ksteps);
                 int e, m, n, s;
-                decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
                 const int kb = s * a.ksteps;
                 const int row = poff[e] + n * BN;
-                for (int ks = 0; ks < a.ksteps; ++ks) {
+                for (int ks = wi.k0; ks < wi.k1; ++ks) {
                     PS_NOW(t0);
                     if (!w.wait(op_empty(st), ph ^ 1u, 2)) goto b_done;
                     PS_ADD(c_bwait, t0);
@@ -235,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             PS_VAR(c_a);
             PS_VAR(c_b);
             PS_VAR(c_issue);
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+            for (int item = blockIdx.x; item < wl.items; item += gridDim.x, ++it) {
+                const WorkItem wi = work_item(wl, item, a.ksteps);
                 const int b = it % C::NDB;
                 const uint32_t aph = (it / C::NDB) & 1;
                 PS_NOW(t0);
@@ -244,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t dcol = tmem_base + b * C::ACC;
                 bool ok = true;
-                for (int ks = 0; ks < a.ksteps; ++ks) {
+                for (int ks = wi.k0; ks < wi.k1; ++ks) {
                     PS_NOW(t1);
                     if (!w.wait(a_full(st), ph, 4)) { ok = false; break; }
                     PS_ADD(c_a, t1);
@@ -266,7 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int kg = (UP ? 0 : bx * (kBKT / 16)) + kk;
                             const uint64_t bdesc =
                                 desc_sw128(bbase + (kg >> 2) * (BN * 128) + (kg & 3) * 32, 16, 1024);
-                            const uint32_t acc = C::DUAL ? ((ks | kk) != 0) : ((ks | bx | kk) != 0);
+                            // the item's first stage starts its accumulator
+                            const int kr = ks - wi.k0;
+                            const uint32_t acc = C::DUAL ? ((kr | kk) != 0) : ((kr | bx | kk) != 0);
                             umma_bf16_ts(dcol + (C::DUAL ? bx : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc,
                                          idesc, acc);
                         }
@@ -295,12 +373,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kCols = BN >= 32 ? BN / 2 : BN;
         const int c0 = BN >= 32 ? hc * kCols : 0;
         const int c1 = BN >= 32 || hc == 0 ? c0 + kCols : c0;
+        volatile uint32_t *last_flag = misc + 2;
+        const EpiOut eo{a.rperm, a.gate, a.h, a.slots, a.M, a.T};
+        auto epilogue_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
         int it = 0;
         PS_VAR(c_ewait);
         PS_VAR(c_ework);
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+        for (int item = blockIdx.x; item < wl.items; item += gridDim.x, ++it) {
+            const WorkItem wi = work_item(wl, item, a.ksteps);
             int e, m, n, s;
-            decode_tile<BN>(tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+            decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
             const int b = it % C::NDB;
             const uint32_t aph = (it / C::NDB) & 1;
             PS_NOW(t0);
@@ -312,55 +394,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = m * kBM + q * 32 + lane;
             const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::ACC;
             const int row0 = poff[e] + n * BN;
-            if constexpr (UP) {
-                const float sa = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
-                const float sb = __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
+            const float sc0 = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
+            const float sc1 = UP ? __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]) : 0.f;
+            const bool whole = wi.piece < 0;   // uniform over the CTA
+            if (!whole) {
+                // a piece: its partial sums go to the workspace, [piece][row][accumulator column]
+                float *pp = a.part + (static_cast<size_t>(wi.piece) * kBM + q * 32 + lane) * C::ACC;
 #pragma unroll 1
                 for (int c = c0; c < c1; c += 16) {
-                    float va[16], vb[16];
+                    float x0[16], x1[16];
                     __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
-                    tmem_ld16(tl + c, va);
-                    tmem_ld16(tl + BN + c, vb);
+                    tmem_ld16(tl + c, x0);
+                    if constexpr (C::NACC == 2) tmem_ld16(tl + BN + c, x1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int r = row0 + c + i;
-                        if (__ldg(a.rperm + r) >= 0)
-                            a.h[static_cast<size_t>(r) * a.M + f] =
-                                __float2bfloat16_rn(gelu_tanh(sa * va[i]) * (sb * vb[i]));
+                    for (int i = 0; i < 16; i += 4) {
+                        *reinterpret_cast<float4 *>(pp + c + i) = make_float4(x0[i], x0[i + 1], x0[i + 2], x0[i + 3]);
+                        if constexpr (C::NACC == 2)
+                            *reinterpret_cast<float4 *>(pp + BN + c + i) =
+                                make_float4(x1[i], x1[i + 1], x1[i + 2], x1[i + 3]);
                     }
                 }
-            } else {
-                const float sc = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty(b));   // the accumulator is no longer needed
+                __threadfence();                             // partial sums before the ticket
+                epilogue_sync();
+                if (warp == kWarpEpi0 && lane == 0) {
+                    unsigned int *tk = a.tickets + (wi.tile - wl.whole);
+                    const bool last = atomicAdd(tk, 1u) == static_cast<unsigned int>(wl.P - 1);
+                    if (last) *tk = 0u;                      // every piece of the tile has arrived
+                    *last_flag = last ? 1u : 0u;
+                }
+                epilogue_sync();
+                if (*last_flag) __threadfence();   // the other pieces' sums, visible after their tickets
+            }
+            if (whole) {
 #pragma unroll 1
                 for (int c = c0; c < c1; c += 16) {
-                    float v[16];
+                    float x0[16], x1[16];
                     __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
-                    tmem_ld16(tl + c, v);
-                    if constexpr (C::DUAL) {   // the two k-box accumulators, summed in this order
-                        float v1[16];
-                        tmem_ld16(tl + BN + c, v1);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] += v1[i];
-                    } else {
-                        tmem_wait_ld();
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int route = __ldg(a.rperm + row0 + c + i);
-                        if (route >= 0) {
-                            const float g = __ldg(a.gate + route);
-                            const size_t o = ((static_cast<size_t>(s) * a.T + (route >> 1)) * 2 + (route & 1)) *
-                                                 static_cast<size_t>(a.M) + f;
-                            a.slots[o] = g * (sc * v[i]);
-                        }
-                    }
+                    tmem_ld16(tl + c, x0);
+                    if constexpr (C::NACC == 2) tmem_ld16(tl + BN + c, x1);
+                    tmem_wait_ld();
+                    epilogue_chunk<UP, C::NACC>(eo, row0, c, f, s, sc0, sc1, x0, x1);
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty(b));
+            } else if (*last_flag) {
+                // the tile's pieces are consecutive in the workspace
+                const float *p0 =
+                    a.part + (static_cast<size_t>(wi.tile - wl.whole) * wl.P * kBM + q * 32 + lane) * C::ACC;
+                finish_pieces<UP, BN, C::NACC, C::ACC>(eo, p0, wl.P, c0, c1, row0, f, s, sc0, sc1);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty(b));
             PS_ADD(c_ework, t1);
         }
         if (lane == 0) {
@@ -387,9 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         PS_VAR(c_cwork);
         PS_VAR(c_cst);
         PS_VAR(c_ctail);
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        for (int item = blockIdx.x; item < wl.items; item += gridDim.x) {
+            const WorkItem wi = work_item(wl, item, a.ksteps);
             bool ok = true;
-            for (int ks = 0; ks < a.ksteps; ++ks) {
+            for (int ks = wi.k0; ks < wi.k1; ++ks) {
                 PS_NOW(t0);
                 ok = __all_sync(0xffffffffu, w.wait(stg_full(st), ph, 7) && w.wait(op_empty(st2), ph2 ^ 1u, 8));
                 if (!ok) break;

@@ -63,6 +63,9 @@ struct GemmArgs {
     float *slots;               // DOWN output [splits, T, 2, M]
     int *err;                   // device error word
     long long timeout_ns;
+    // last-wave pieces (TMEM-operand kernels): partial accumulators and per-tile tickets
+    float *part;                // [gridDim.x, 128, accumulator columns] fp32, or nullptr: no pieces
+    unsigned int *tickets;      // [gridDim.x], zero, left zero by every launch that completes
 };
 
 struct CombineArgs {

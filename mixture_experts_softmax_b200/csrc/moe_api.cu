@@ -49,7 +49,10 @@ struct moe_ctx {
     DevBuf b_h;        // bf16 [rows, F]
     DevBuf b_slots;    // fp32 [splits, T, 2, d]
     DevBuf b_stage;    // bf16 [T, d] x2: host-API input/output staging, block pre-norm output
-    int *err = nullptr;     // 256 zeroed bytes: word 0 the device error word, word 32 the routing ticket
+    // kCtlWords zeroed words: [0] the device error word, [32] the routing ticket, [64 ..) the
+    // GEMMs' last-wave tickets (one per SM)
+    int *err = nullptr;
+    DevBuf b_part;     // fp32 [num_sms, 128, 256]: the GEMMs' last-wave partial sums
     int rows_cap = 0;       // rows the xp / h buffers hold
     int route_cap = 0;      // T the route buffer holds
     int map_gen = 0;        // bumps when b_xp / b_h move
@@ -71,6 +74,10 @@ struct moe_ctx {
 };
 
 namespace {
+
+constexpr int kCtlWords = 1024;     // words of the handle's zeroed control block
+constexpr int kCtlRouteTicket = 32;
+constexpr int kCtlTickets = 64;     // first GEMM ticket
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -173,11 +180,12 @@ int ensure_device(moe_ctx *h)
         if (p.major != 10) return MOE_ENODEV;   // built for sm_100a only
         h->device = dev;
         h->num_sms = p.multiProcessorCount;
-        if (cudaMalloc(reinterpret_cast<void **>(&h->err), 256) != cudaSuccess) {
+        if (h->num_sms + kCtlTickets > kCtlWords) return MOE_EUNSUPPORTED;
+        if (cudaMalloc(reinterpret_cast<void **>(&h->err), kCtlWords * 4) != cudaSuccess) {
             cudaGetLastError();
             return MOE_ENOMEM;
         }
-        if (cudaMemset(h->err, 0, 256) != cudaSuccess) return MOE_ECUDA;
+        if (cudaMemset(h->err, 0, kCtlWords * 4) != cudaSuccess) return MOE_ECUDA;
     } else if (dev != h->device) {
         return MOE_EINVAL;   // the handle belongs to another device
     }
@@ -202,6 +210,10 @@ int ensure_workspace(moe_ctx *h, int T, int bn, int splits)
     (void)moved;
     if ((rc = ensure(h, h->b_slots, static_cast<size_t>(splits) * T * 2 * h->d * 4)) != MOE_OK) return rc;
     if ((rc = ensure(h, h->b_stage, static_cast<size_t>(T) * h->d * 2 * 2)) != MOE_OK) return rc;
+    // last-wave partial sums of the TMEM GEMMs: one 128-row tile of up to 256 fp32 columns per SM
+    if (h->layout == MOE_LAYOUT_PACKED &&
+        (rc = ensure(h, h->b_part, static_cast<size_t>(h->num_sms) * 128 * 256 * 4)) != MOE_OK)
+        return rc;
     return MOE_OK;
 }
 
@@ -359,7 +371,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     DispatchArgs da{T, h->E, bn, idx, rw + L.counts, rw + L.offsets, poff, rw + L.perm, rperm, rw + L.slot};
     GatherArgs ga{h->d, static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
     if (T <= route_small_max_tokens()) {
-        unsigned int *ticket = reinterpret_cast<unsigned int *>(h->err + 32);
+        unsigned int *ticket = reinterpret_cast<unsigned int *>(h->err + kCtlRouteTicket);
         if (timed(h, K_ROUTE_SMALL, s, [&] { return launch_route_small(ra, da, ga, ticket, s); }) != cudaSuccess)
             return MOE_ECUDA;
     } else {
@@ -384,6 +396,10 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.h = static_cast<__nv_bfloat16 *>(h->b_h.ptr);
     up.err = h->err;
     up.timeout_ns = h->timeout_ns;
+    if (ts) {
+        up.part = static_cast<float *>(h->b_part.ptr);
+        up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
+    }
     if (timed(h, K_UP, s, [&] {
             return ts ? launch_gemm_up_ts(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s)
                       : launch_gemm_up(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s);
@@ -471,6 +487,7 @@ MOE_API int moe_destroy(moe_handle h)
     for (DevBuf *b : {&h->b_route, &h->b_rperm, &h->b_xp, &h->b_h, &h->b_slots, &h->b_stage})
         if (b->ptr) cudaFree(b->ptr);
     if (h->err) cudaFree(h->err);
+    if (h->b_part.ptr) cudaFree(h->b_part.ptr);
     for (auto &p : h->pending) {
         cudaEventDestroy(p.a);
         cudaEventDestroy(p.b);
@@ -609,7 +626,8 @@ MOE_API int moe_sync_status(moe_handle h, void *stream)
     int e = 0;
     if (cudaMemcpy(&e, h->err, sizeof e, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ECUDA;
     if (e == 0) return MOE_OK;
-    cudaMemset(h->err, 0, sizeof e);
+    // a kernel that gave up may have left tickets taken: clear the whole control block
+    cudaMemset(h->err, 0, kCtlWords * 4);
     return e >= kErrTimeoutBase ? MOE_ETIMEOUT : MOE_ECUDA;
 }
 
