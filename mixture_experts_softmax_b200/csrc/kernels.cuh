@@ -24,6 +24,11 @@ struct RouteArgs {
     const float *bias;          // [E] or nullptr
     int *idx;                   // [T, 2]
     float *gate;                // [T, 2]
+    // optional pre-MoE RMSNorm (small-batch routing only): route on u = bf16(x * rsqrt(mean x^2 + eps) * g),
+    // written to u for the gather
+    const __nv_bfloat16 *g_pre; // [d] or nullptr
+    float eps;
+    __nv_bfloat16 *u;           // [T, d]
 };
 
 struct DispatchArgs {

@@ -348,7 +348,7 @@ int check_weights(const moe_ctx *h, const float *router_w, const int8_t *w_lin, 
 // the layer on x (device, bf16 [T, d]); result into `out` (plain) or added into h_io (residual block)
 int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int8_t *w_lin, const void *s_lin,
               const int8_t *w_v, const void *s_v, const int8_t *w_1, const void *s_1, void *out, void *h_io,
-              const void *g_post, float eps, cudaStream_t s)
+              const void *g_pre, const void *g_post, float eps, cudaStream_t s)
 {
     int rc;
     const int bn = plan_bn(T);
@@ -367,10 +367,25 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     if ((rc = weight_map(h, w_1, 1, &m_w1)) != MOE_OK) return rc;
     if ((rc = act_maps(h, bn, &m_xp, &m_h)) != MOE_OK) return rc;
 
-    RouteArgs ra{T, h->d, static_cast<const __nv_bfloat16 *>(x), router_w, h->bias, idx, gate};
+    // residual block: the routed rows are u = pre-RMSNorm(x), in the staging buffer; small
+    // batches normalise inside the routing launch, larger ones in a pre-norm launch first
+    const bool small = T <= route_small_max_tokens();
+    __nv_bfloat16 *u = static_cast<__nv_bfloat16 *>(h->b_stage.ptr);
+    const __nv_bfloat16 *routed = static_cast<const __nv_bfloat16 *>(x);
+    if (g_pre && !small) {
+        NormArgs na{T, h->d, routed, static_cast<const __nv_bfloat16 *>(g_pre), eps, u};
+        if (timed(h, K_PRENORM, s, [&] { return launch_prenorm(na, s); }) != cudaSuccess) return MOE_ECUDA;
+        routed = u;
+    }
+    RouteArgs ra{T, h->d, routed, router_w, h->bias, idx, gate};
+    if (g_pre && small) {
+        ra.g_pre = static_cast<const __nv_bfloat16 *>(g_pre);
+        ra.eps = eps;
+        ra.u = u;
+    }
     DispatchArgs da{T, h->E, bn, idx, rw + L.counts, rw + L.offsets, poff, rw + L.perm, rperm, rw + L.slot};
-    GatherArgs ga{h->d, static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
-    if (T <= route_small_max_tokens()) {
+    GatherArgs ga{h->d, g_pre ? u : routed, static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
+    if (small) {
         unsigned int *ticket = reinterpret_cast<unsigned int *>(h->err + kCtlRouteTicket);
         if (timed(h, K_ROUTE_SMALL, s, [&] { return launch_route_small(ra, da, ga, ticket, s); }) != cudaSuccess)
             return MOE_ECUDA;
@@ -555,7 +570,7 @@ MOE_API int moe_forward(moe_handle h, int T, const void *x, const float *router_
     if (overlaps(x, xb, out, xb)) return MOE_EINVAL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((rc = begin_call(h, T, s)) != MOE_OK) return rc;
-    return run_layer(h, T, x, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, out, nullptr, nullptr, 0.f, s);
+    return run_layer(h, T, x, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, out, nullptr, nullptr, nullptr, 0.f, s);
 }
 
 MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const float *router_w, const int8_t *w_lin,
@@ -573,7 +588,8 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
     char *xs = static_cast<char *>(h->b_stage.ptr);
     char *os = xs + xb;
     if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ECUDA;
-    if ((rc = run_layer(h, T, xs, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, os, nullptr, nullptr, 0.f, s)) != MOE_OK)
+    if ((rc = run_layer(h, T, xs, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, os, nullptr, nullptr, nullptr, 0.f, s)) !=
+        MOE_OK)
         return rc;
     if (cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
     return MOE_OK;
@@ -591,10 +607,7 @@ MOE_API int moe_block_forward(moe_handle h, int T, void *h_io, const void *g_pre
     if (rc != MOE_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((rc = begin_call(h, T, s)) != MOE_OK) return rc;
-    __nv_bfloat16 *u = static_cast<__nv_bfloat16 *>(h->b_stage.ptr);
-    NormArgs na{T, h->d, static_cast<const __nv_bfloat16 *>(h_io), static_cast<const __nv_bfloat16 *>(g_pre), eps, u};
-    if (timed(h, K_PRENORM, s, [&] { return launch_prenorm(na, s); }) != cudaSuccess) return MOE_ECUDA;
-    return run_layer(h, T, u, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, nullptr, h_io, g_post, eps, s);
+    return run_layer(h, T, h_io, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, nullptr, h_io, g_pre, g_post, eps, s);
 }
 
 MOE_API int moe_get_routing(moe_handle h, int32_t *idx, float *gate, int32_t *offsets, int32_t *perm, void *stream)

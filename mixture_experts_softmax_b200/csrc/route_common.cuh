@@ -62,7 +62,10 @@ constexpr int kRouteTokenThreads = 256;
 // The logits of token t by one block of kRouteTokenThreads threads splitting d: every
 // thread issues all its loads at once (one memory latency), then a fixed-order reduction
 // (lane tree, then the warp partials in warp order) gives the logits; thread 0 writes the
-// token's top-2 experts and gates.
+// token's top-2 experts and gates.  With a.g_pre set, the routed row is the RMS-normalised
+// u = bf16(x * rsqrt(mean(x^2) + eps) * g) of the residual block, which is also written to
+// a.u: the sum of squares is reduced first (same fixed order), then every 8-element chunk
+// of u is formed in fp32, rounded to bf16, stored and used.
 __device__ __forceinline__ void route_token(const RouteArgs &a, int t)
 {
     constexpr int kWarps = kRouteTokenThreads / 32;
@@ -70,12 +73,51 @@ __device__ __forceinline__ void route_token(const RouteArgs &a, int t)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * a.d);
     const float4 *w4 = reinterpret_cast<const float4 *>(a.w);
+    const int chunks = a.d >> 3;
     float acc[kExperts];
 #pragma unroll
     for (int e = 0; e < kExperts; ++e) acc[e] = 0.f;
-    const int chunks = a.d >> 3;
+    if (a.g_pre) {
+        float ss = 0.f;
+        for (int c = threadIdx.x; c < chunks; c += kRouteTokenThreads) {
+            const uint4 v = __ldg(xr + c);
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float lo = __uint_as_float(wv[q] << 16), hi = __uint_as_float(wv[q] & 0xffff0000u);
+                ss = fmaf(lo, lo, ss);
+                ss = fmaf(hi, hi, ss);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) part[warp][0] = ss;
+        __syncthreads();
+        float tot = 0.f;
+        for (int w = 0; w < kWarps; ++w) tot += part[w][0];
+        __syncthreads();   // part is reused for the logits below
+        const float r = rsqrtf(tot / static_cast<float>(a.d) + a.eps);
+        const uint4 *gr = reinterpret_cast<const uint4 *>(a.g_pre);
+        uint4 *ur = reinterpret_cast<uint4 *>(a.u + static_cast<size_t>(t) * a.d);
+        for (int c = threadIdx.x; c < chunks; c += kRouteTokenThreads) {
+            const uint4 v = __ldg(xr + c), g = __ldg(gr + c);
+            const uint32_t hv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w};
+            uint32_t uv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float lo = __uint_as_float(hv[q] << 16) * r * __uint_as_float(gv[q] << 16);
+                const float hi = __uint_as_float(hv[q] & 0xffff0000u) * r * __uint_as_float(gv[q] & 0xffff0000u);
+                const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+                uv[q] = *reinterpret_cast<const uint32_t *>(&p);
+            }
+            const uint4 u = make_uint4(uv[0], uv[1], uv[2], uv[3]);
+            ur[c] = u;
+            dot8(u, w4, c * 8, acc);
+        }
+    } else {
 #pragma unroll 4
-    for (int c = threadIdx.x; c < chunks; c += kRouteTokenThreads) dot8(__ldg(xr + c), w4, c * 8, acc);
+        for (int c = threadIdx.x; c < chunks; c += kRouteTokenThreads) dot8(__ldg(xr + c), w4, c * 8, acc);
+    }
 #pragma unroll
     for (int e = 0; e < kExperts; ++e) {
 #pragma unroll

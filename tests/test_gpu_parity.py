@@ -140,6 +140,39 @@ def test_small_batch_routing_is_one_launch(m, tiny_inputs, tiny_handle):
         assert times[k][1] == 0
 
 
+@pytest.mark.parametrize("T", [8, 64])
+def test_tiny_residual_block(m, tiny_inputs, tiny_handle, T):
+    """moe_block_forward on the tiny layer with non-unit RMSNorm gains: T=8 takes the
+    pre-norm inside the small-batch routing launch, T=64 the separate pre-norm kernel."""
+    h, layer, _ = tiny_handle
+    layer_cpu = parity.to_cpu(tiny_inputs.layers[0])
+    g = torch.Generator().manual_seed(11)
+    gam = {k: (0.5 + torch.rand(256, generator=g)).to(torch.bfloat16) for k in ("pre", "post")}
+    h_in = tiny_inputs.x[:T].clone()
+    chain = oracle.block_chain([layer_cpu], [gam], h_in, eps=1e-5)[0]
+    h_dev = h_in.cuda().contiguous()
+    m.check(m.moe_set_router_bias(h, None))
+    m.check(m.moe_block_forward(h, T, h_dev, gam["pre"].cuda(), gam["post"].cuda(), 1e-5, *m.layer_args(layer)))
+    idx = torch.empty((T, 2), dtype=torch.int32, device="cuda")
+    m.check(m.moe_get_routing(h, idx))
+    m.check(m.moe_sync_status(h))
+    gidx = idx.cpu().numpy()
+    diff = (gidx != chain["idx"]).any(axis=1)
+    ref_out = chain["h_out"]
+    if diff.any():
+        # the bf16 routed row can round differently after an fp32 vs fp64 RMSNorm; such a
+        # token must be a close call in the oracle, and is compared with the GPU's experts
+        srt = -np.sort(-chain["probs"], axis=1)
+        gap = np.minimum(srt[:, 0] - srt[:, 1], srt[:, 1] - srt[:, 2])
+        assert (gap[diff] < 1e-4).all(), f"routing differs on {np.nonzero(diff)[0]}"
+        forced = [gidx[t] if diff[t] else chain["idx"][t] for t in range(T)]
+        ref_out = oracle.block_chain([layer_cpu], [gam], h_in, eps=1e-5, forced=[np.array(forced)])[0]["h_out"]
+    got = h_dev.cpu().to(torch.float64).numpy()
+    dg, dr = got - chain["h_in"], ref_out - chain["h_in"]
+    err = np.abs(dg - dr).max()
+    assert err <= parity.OUT_RTOL * np.abs(dr).max() + 2 * np.abs(ref_out).max() * 2.0 ** -8, err
+
+
 def test_pack_weight_is_a_transpose(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
