@@ -118,7 +118,7 @@ __device__ __forceinline__ void decode_tile(int tile, const int *prefix, const i
 // (stream-K for the last wave only), so every CTA runs the same number of whole tiles and
 // at most one piece.  A piece leaves its fp32 accumulator in a workspace; the piece that
 // finishes last (a ticket per tile) adds the P partial sums in piece order and applies the
-// tile's epilogue.  P < 2 means no pieces.
+// tile's epilogue.  P < 2 means no pieces; so do fewer tiles than CTAs (test-sized problems).
 struct WorkList {
     int whole;    // items [0, whole): whole tiles 0 .. whole-1
     int P;        // pieces per split tile
@@ -131,7 +131,7 @@ __device__ __forceinline__ WorkList make_work_list(int tiles, int grid, int kste
     const int r = tiles % grid;
     int P = r ? grid / r : 0;
     if (P > ksteps) P = ksteps;
-    if (P < 2) P = 0;
+    if (P < 2 || tiles < grid) P = 0;   // pieces only behind at least one full wave of whole tiles
     q.P = P;
     q.whole = P ? tiles - r : tiles;
     q.items = q.whole + (P ? r * P : 0);
