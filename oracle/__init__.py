@@ -74,7 +74,7 @@ def lib():
         L.moe_oracle_expert_ffn.restype = i
         L.moe_oracle_expert_ffn.argtypes = [i, i, P, P, P, P, P, P, P, P, P, i, i]
         L.moe_oracle_forward.restype = i
-        L.moe_oracle_forward.argtypes = [i, i, i, i, P, P, P, P, P, P, P, P, P, P, i, P, P, P, P, i, i]
+        L.moe_oracle_forward.argtypes = [i, i, i, i, P, P, P, P, P, P, P, P, P, P, i, P, P, P, P, P, i, i]
         L.moe_oracle_rmsnorm.restype = i
         L.moe_oracle_rmsnorm.argtypes = [i, i, P, P, ctypes.c_double, P]
         _lib = L
@@ -165,7 +165,10 @@ def route(x, router_w, bias=None) -> Dict[str, np.ndarray]:
 
 
 def dispatch(idx, E: int):
-    """counts [E], offsets [E+1], perm [2T] (route id 2t+j), grouped by expert, stable in t."""
+    """counts [E], offsets [E+1], perm [2T] (route id 2t+j), grouped by expert, stable in t.
+
+    Expert id -1 (a padding token's route) is not dispatched; perm entries from offsets[E]
+    on are then unused (0)."""
     ia = _np(idx, np.int32)
     T = ia.shape[0]
     counts = np.zeros(E, np.int32)
@@ -192,8 +195,11 @@ def expert_ffn(xt: np.ndarray, layer, e: int, nthreads: int = 0, gelu_kind: int 
 
 
 def forward(layer, x, bias=None, tokens: Optional[Sequence[int]] = None, forced_idx=None,
-            nthreads: int = 0, gelu_kind: int = 0):
-    """The MoE layer on the selected tokens: returns (out fp64 [n,d], idx [n,2], gate [n,2])."""
+            nthreads: int = 0, gelu_kind: int = 0, mask=None):
+    """The MoE layer on the selected tokens: returns (out fp64 [n,d], idx [n,2], gate [n,2]).
+
+    ``mask`` (bool/uint8 [T], optional): tokens with mask 0 are padding, routed nowhere
+    (out row 0, experts -1, gates 0)."""
     xb = _np(x, np.uint16)
     T, d = xb.shape
     rw = _np(layer["router_w"], np.float32)
@@ -207,11 +213,14 @@ def forward(layer, x, bias=None, tokens: Optional[Sequence[int]] = None, forced_
     fi = None if forced_idx is None else np.ascontiguousarray(np.asarray(forced_idx, dtype=np.int32))
     if fi is not None and fi.shape != (n, 2):
         raise ValueError("forced_idx must be [n_sel, 2]")
+    mk = None if mask is None else np.ascontiguousarray(_np(mask).astype(np.uint8).reshape(-1))
+    if mk is not None and mk.shape[0] != T:
+        raise ValueError("mask must have one entry per token")
     out = np.zeros((n, d), np.float64)
     idx = np.zeros((n, 2), np.int32)
     gate = np.zeros((n, 2), np.float64)
     _check(lib().moe_oracle_forward(T, d, F, E, _p(xb), _p(rw), _p(b), _p(wl), _p(sl), _p(wv),
-                                    _p(sv), _p(w1), _p(s1), _p(tk), n, _p(fi), _p(out), _p(idx),
+                                    _p(sv), _p(w1), _p(s1), _p(tk), n, _p(fi), _p(mk), _p(out), _p(idx),
                                     _p(gate), nthreads, gelu_kind), "forward")
     return out, idx, gate
 
@@ -238,7 +247,7 @@ def near_ties(probs: np.ndarray, thresh: float = 1e-6) -> np.ndarray:
 
 def block_chain(layers: List[dict], gammas: List[dict], h, eps: float = 1e-5,
                 tokens: Optional[Sequence[int]] = None, forced: Optional[List[Optional[np.ndarray]]] = None,
-                nthreads: int = 0, gelu_kind: int = 0):
+                nthreads: int = 0, gelu_kind: int = 0, mask=None):
     """Stacked residual MoE blocks on the selected token rows of h (bf16 [T,d]).
 
     Per block b:  u = bf16( RMSNorm(h; g_pre) )        (the MoE layer's bf16 input)
@@ -246,11 +255,14 @@ def block_chain(layers: List[dict], gammas: List[dict], h, eps: float = 1e-5,
                   h = bf16( h + RMSNorm(y; g_post) )    (bf16 residual stream)
     Returns a list of per-block dicts: h_in (fp64 values of bf16), u, idx, gate, probs, h_out.
     ``forced[b]`` (optional [n,2]) names the experts to use in block b.
+    ``mask`` (optional [T]) marks padding tokens (0): their MoE output is 0, so their row of
+    the residual stream passes through unchanged.
     """
     hb = _np(h, np.uint16)
     T, d = hb.shape
     rows = list(range(T)) if tokens is None else [int(t) for t in tokens]
     cur = bf16_bits_to_f64(hb[rows])
+    mk = None if mask is None else np.asarray(_np(mask)).astype(np.uint8).reshape(-1)[rows]
     res = []
     for b, (layer, gm) in enumerate(zip(layers, gammas)):
         u = round_bf16(rmsnorm(cur, gm["pre"], eps))
@@ -258,7 +270,7 @@ def block_chain(layers: List[dict], gammas: List[dict], h, eps: float = 1e-5,
         r = route(ub, layer["router_w"])
         fb = None if forced is None else forced[b]
         y, idx, gate = forward(layer, ub, tokens=None, forced_idx=fb, nthreads=nthreads,
-                               gelu_kind=gelu_kind)
+                               gelu_kind=gelu_kind, mask=mk)
         nxt = round_bf16(cur + rmsnorm(y, gm["post"], eps))
         res.append(dict(h_in=cur, u=u, idx=idx, gate=gate, probs=r["probs"], h_out=nxt))
         cur = nxt

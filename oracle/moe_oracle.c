@@ -189,6 +189,7 @@ ORACLE_API int moe_oracle_dispatch(int T, int E, const int32_t *idx, int32_t *co
     for (int t = 0; t < T; ++t)
         for (int j = 0; j < 2; ++j) {
             int e = idx[2 * t + j];
+            if (e == -1) continue;   /* a padding token's route: not dispatched */
             if (e < 0 || e >= E) { free(cnt); return OR_EINVAL; }
             cnt[e]++;
         }
@@ -200,7 +201,7 @@ ORACLE_API int moe_oracle_dispatch(int T, int E, const int32_t *idx, int32_t *co
         for (int t = 0; t < T; ++t)
             for (int j = 0; j < 2; ++j) {
                 int e = idx[2 * t + j];
-                perm[offsets[e] + cnt[e]++] = 2 * t + j;
+                if (e >= 0) perm[offsets[e] + cnt[e]++] = 2 * t + j;
             }
     }
     free(cnt);
@@ -337,14 +338,18 @@ ORACLE_API int moe_oracle_expert_ffn(int d, int F, const double *xt, const int8_
  * forced_idx (int32 [n_sel,2], may be NULL) names the two experts to use; the
  * gates are then those experts' softmax probabilities.
  * Weights: wl, wv int8 [E,d,F], w1 int8 [E,F,d]; sl, sv bf16 [E,F]; s1 bf16 [E,d].
+ * mask (uint8 [T], may be NULL = every token real): a token t with mask[t] == 0 is
+ * padding, the padding_mask of the MoE call in the grok-field-guide source-code map,
+ * fourth stop (moe(rms_norm(h), padding_mask)); it is routed nowhere: out row 0,
+ * experts -1 and gates 0.
  * Outputs: out fp64 [n_sel,d]; idx int32 [n_sel,2] and gate fp64 [n_sel,2] (may be NULL).
  */
 ORACLE_API int moe_oracle_forward(int T, int d, int F, int E, const uint16_t *x,
                                   const float *router_w, const float *bias, const int8_t *wl,
                                   const uint16_t *sl, const int8_t *wv, const uint16_t *sv,
                                   const int8_t *w1, const uint16_t *s1, const int32_t *tokens,
-                                  int n_sel, const int32_t *forced_idx, double *out, int32_t *idx,
-                                  double *gate, int nthreads, int gelu_kind)
+                                  int n_sel, const int32_t *forced_idx, const uint8_t *mask, double *out,
+                                  int32_t *idx, double *gate, int nthreads, int gelu_kind)
 {
     if (T < 0 || d <= 0 || F <= 0 || E < 2 || E > 64 || !x || !router_w || !wl || !sl || !wv ||
         !sv || !w1 || !s1 || !out)
@@ -359,6 +364,12 @@ ORACLE_API int moe_oracle_forward(int T, int d, int F, int E, const uint16_t *x,
         int t = tokens ? tokens[s] : s;
         if (t < 0 || t >= T) { rc = OR_EINVAL; break; }
         const uint16_t *xrow = x + (size_t)t * d;
+        if (mask && !mask[t]) {
+            for (int i = 0; i < d; ++i) out[(size_t)s * d + i] = 0.0;
+            if (idx) { idx[2 * s] = -1; idx[2 * s + 1] = -1; }
+            if (gate) { gate[2 * s] = 0.0; gate[2 * s + 1] = 0.0; }
+            continue;
+        }
         int32_t sel[2];
         rc = moe_oracle_route(1, d, E, xrow, router_w, bias, NULL, probs, sel, NULL);
         if (rc != OR_OK) break;

@@ -170,6 +170,22 @@ def test_dispatch_brute_force():
         assert perm.tolist() == [r for gr in groups for r in gr]
 
 
+def test_dispatch_skips_padding_routes():
+    """Expert id -1 (a padding token) is not dispatched: brute-force grouping of the rest."""
+    g = torch.Generator().manual_seed(12)
+    E, T = 8, 200
+    idx = np.zeros((T, 2), np.int32)
+    for t in range(T):
+        idx[t] = torch.randperm(E, generator=g)[:2].numpy()
+    pad = (torch.rand(T, generator=g) < 0.3).numpy()
+    idx[pad] = -1
+    counts, offsets, perm = oracle.dispatch(idx, E)
+    groups = [[2 * t + j for t in range(T) for j in range(2) if idx[t, j] == e] for e in range(E)]
+    assert counts.tolist() == [len(gr) for gr in groups]
+    assert offsets[-1] == 2 * int((~pad).sum())
+    assert perm[:offsets[-1]].tolist() == [r for gr in groups for r in gr]
+
+
 # ---- expert FFN and the layer -------------------------------------------------
 
 def test_expert_ffn_matches_numpy(tiny):
@@ -251,6 +267,26 @@ def test_zero_input_gives_zero_output(tiny):
     assert np.all(out == 0.0)
     assert (idx == [[0, 1]] * 4).all()
     assert np.all(gate == 0.125)
+
+
+def test_padding_mask_routes_nothing(tiny):
+    """Padding tokens get output 0, experts -1, gates 0; every real token's result is
+    bit-identical to the unmasked layer's (tokens are independent)."""
+    layer = tiny.layers[0]
+    g = torch.Generator().manual_seed(8)
+    mask = (torch.rand(tiny.x.shape[0], generator=g) > 0.3).numpy()
+    out, idx, gate = oracle.forward(layer, tiny.x)
+    out_m, idx_m, gate_m = oracle.forward(layer, tiny.x, mask=mask)
+    assert np.array_equal(out_m[mask], out[mask])
+    assert np.array_equal(idx_m[mask], idx[mask]) and np.array_equal(gate_m[mask], gate[mask])
+    assert np.all(out_m[~mask] == 0.0) and (idx_m[~mask] == -1).all() and np.all(gate_m[~mask] == 0.0)
+    out_0, idx_0, _ = oracle.forward(layer, tiny.x[:5], mask=np.zeros(5, np.uint8))
+    assert np.all(out_0 == 0.0) and (idx_0 == -1).all()
+    # in the residual block a padding row passes through unchanged
+    gam = {"pre": torch.ones(tiny.x.shape[1], dtype=torch.bfloat16),
+           "post": torch.ones(tiny.x.shape[1], dtype=torch.bfloat16)}
+    blk = oracle.block_chain([layer], [gam], tiny.x[:16], mask=mask[:16])[0]
+    assert np.array_equal(blk["h_out"][~mask[:16]], blk["h_in"][~mask[:16]])
 
 
 def test_linear_in_output_scale(tiny):
