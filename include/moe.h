@@ -103,6 +103,19 @@ MOE_API int moe_destroy(moe_handle h);
 MOE_API int moe_set_router_bias(moe_handle h, const float *bias);
 
 /*
+ * Padding mask of the MoE call: the grok-field-guide source-code map, fourth stop,
+ * passes one to the layer (moe(rms_norm(h), padding_mask)).  mask: device uint8
+ * [T] (one byte per token: nonzero = a real token, 0 = padding), or NULL for "every
+ * token real".  A padding token is routed nowhere: moe_get_routing reports experts
+ * -1 and gates 0 for it, the dispatch skips its routes, its output row of
+ * moe_forward / moe_forward_host is 0 and moe_block_forward leaves its residual
+ * row unchanged.  The pointer is kept, not copied: it must hold at least T bytes
+ * for every later forward on this handle and stay valid while they run.
+ * Errors: MOE_EINVAL for a NULL handle.
+ */
+MOE_API int moe_set_padding_mask(moe_handle h, const uint8_t *mask);
+
+/*
  * The MoE layer on T tokens ("Mixture of Experts (MoELayer + Router)", steps 1-4).
  *   x    bf16 [T, d]   input tokens
  *   out  bf16 [T, d]   output; must not overlap x or the weights

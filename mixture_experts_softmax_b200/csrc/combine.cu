@@ -42,7 +42,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
         const int t = static_cast<int>(i / per_row), c = static_cast<int>(i % per_row) * 4;
-        const float4 y = slot_sum(a, t, c);
+        // a padding token (expert -1) has no slots: its output row is 0
+        const float4 y = __ldg(a.idx + 2 * t) < 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : slot_sum(a, t, c);
         __nv_bfloat162 lo = __floats2bfloat162_rn(y.x, y.y), hi = __floats2bfloat162_rn(y.z, y.w);
         uint2 v;
         v.x = *reinterpret_cast<uint32_t *>(&lo);
@@ -56,6 +57,7 @@ __global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
 {
     __shared__ float red[8];
     const int t = blockIdx.x;
+    if (__ldg(a.idx + 2 * t) < 0) return;   // a padding token: the residual row passes through unchanged
     float ss = 0.f;
     for (int c = threadIdx.x * 4; c < a.d; c += blockDim.x * 4) {
         const float4 y = slot_sum(a, t, c);

@@ -34,9 +34,10 @@ __device__ __forceinline__ void dispatch_block(const DispatchArgs &a)
     const int E = a.E;
     if (tid < kMaxE) { s_cnt[tid] = 0; s_run[tid] = 0; }
     __syncthreads();
-    for (int t = tid; t < a.T; t += NT) {
-        atomicAdd(&s_cnt[__ldcg(a.idx + 2 * t)], 1);
-        atomicAdd(&s_cnt[__ldcg(a.idx + 2 * t + 1)], 1);
+    for (int t = tid; t < a.T; t += NT) {   // expert -1: a padding token's route, not dispatched
+        const int e0 = __ldcg(a.idx + 2 * t), e1 = __ldcg(a.idx + 2 * t + 1);
+        if (e0 >= 0) atomicAdd(&s_cnt[e0], 1);
+        if (e1 >= 0) atomicAdd(&s_cnt[e1], 1);
     }
     __syncthreads();
     if (tid == 0) {
@@ -81,13 +82,20 @@ __device__ __forceinline__ void dispatch_block(const DispatchArgs &a)
         }
         if (valid) {
             const int r0 = 2 * t, r1 = 2 * t + 1;
-            a.perm[s_off[e0] + rank0] = r0;
-            a.perm[s_off[e1] + rank1] = r1;
-            const int p0 = s_poff[e0] + rank0, p1 = s_poff[e1] + rank1;
-            a.rperm[p0] = r0;
-            a.rperm[p1] = r1;
-            a.slot_of_route[r0] = p0;
-            a.slot_of_route[r1] = p1;
+            if (e0 >= 0) {
+                a.perm[s_off[e0] + rank0] = r0;
+                a.rperm[s_poff[e0] + rank0] = r0;
+                a.slot_of_route[r0] = s_poff[e0] + rank0;
+            } else {
+                a.slot_of_route[r0] = -1;
+            }
+            if (e1 >= 0) {
+                a.perm[s_off[e1] + rank1] = r1;
+                a.rperm[s_poff[e1] + rank1] = r1;
+                a.slot_of_route[r1] = s_poff[e1] + rank1;
+            } else {
+                a.slot_of_route[r1] = -1;
+            }
         }
         __syncthreads();   // s_warp is rewritten by the next chunk
     }
@@ -121,10 +129,11 @@ __device__ __forceinline__ void gather_rows(const GatherArgs &g, int T, const in
                 if (u < n) v[u] = __ldg(reinterpret_cast<const uint4 *>(g.x + static_cast<size_t>(t0 + u) * g.d) + c);
 #pragma unroll
             for (int u = 0; u < kGatherTokens; ++u) {
-                if (u < n) {
+                if (u < n) {   // slot -1: a padding token's route
                     const int r = 2 * (t0 + u);
-                    reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(slot_of_route[r]) * g.d)[c] = v[u];
-                    reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(slot_of_route[r + 1]) * g.d)[c] = v[u];
+                    const int p0 = slot_of_route[r], p1 = slot_of_route[r + 1];
+                    if (p0 >= 0) reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(p0) * g.d)[c] = v[u];
+                    if (p1 >= 0) reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(p1) * g.d)[c] = v[u];
                 }
             }
         }

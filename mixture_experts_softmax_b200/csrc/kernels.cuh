@@ -29,6 +29,7 @@ struct RouteArgs {
     const __nv_bfloat16 *g_pre; // [d] or nullptr
     float eps;
     __nv_bfloat16 *u;           // [T, d]
+    const uint8_t *mask;        // [T] padding mask (0 = padding: experts -1, gates 0) or nullptr
 };
 
 struct DispatchArgs {
@@ -76,6 +77,7 @@ struct GemmArgs {
 struct CombineArgs {
     int T, d, splits;
     const float *slots;         // [splits, T, 2, d]
+    const int *idx;             // [T, 2] experts; -1: a padding token (no slots written), output 0
     __nv_bfloat16 *out;         // [T, d]
     // residual block variant
     __nv_bfloat16 *h_io;        // [T, d] residual stream (nullptr: plain combine)

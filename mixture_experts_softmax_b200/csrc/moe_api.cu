@@ -64,6 +64,7 @@ struct moe_ctx {
     int xp_map_gen[4] = {-1, -1, -1, -1}, h_map_gen[4] = {-1, -1, -1, -1};
 
     const float *bias = nullptr;
+    const uint8_t *mask = nullptr;   // padding mask of the next forwards (device, >= T bytes)
     long long timeout_ns = 2000000000LL;
     int layout = MOE_LAYOUT_IN_OUT;
 
@@ -378,6 +379,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
         routed = u;
     }
     RouteArgs ra{T, h->d, routed, router_w, h->bias, idx, gate};
+    ra.mask = h->mask;
     if (g_pre && small) {
         ra.g_pre = static_cast<const __nv_bfloat16 *>(g_pre);
         ra.eps = eps;
@@ -436,7 +438,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
         }) != cudaSuccess)
         return MOE_ECUDA;
 
-    CombineArgs ca{T, h->d, splits, static_cast<const float *>(h->b_slots.ptr), static_cast<__nv_bfloat16 *>(out),
+    CombineArgs ca{T, h->d, splits, static_cast<const float *>(h->b_slots.ptr), idx, static_cast<__nv_bfloat16 *>(out),
                    static_cast<__nv_bfloat16 *>(h_io), static_cast<const __nv_bfloat16 *>(g_post), eps};
     if (timed(h, K_COMBINE, s, [&] { return launch_combine(ca, s); }) != cudaSuccess) return MOE_ECUDA;
     h->last_T = T;
@@ -517,6 +519,13 @@ MOE_API int moe_set_router_bias(moe_handle h, const float *bias)
     if (!h) return MOE_EINVAL;
     if (bias && !aligned16(bias)) return MOE_EINVAL;
     h->bias = bias;
+    return MOE_OK;
+}
+
+MOE_API int moe_set_padding_mask(moe_handle h, const uint8_t *mask)
+{
+    if (!h) return MOE_EINVAL;
+    h->mask = mask;
     return MOE_OK;
 }
 

@@ -59,6 +59,17 @@ __device__ __forceinline__ void select_top2(float (&acc)[kExperts], const float 
 
 constexpr int kRouteTokenThreads = 256;
 
+// a padding token (padding mask 0) is routed nowhere: experts -1, gates 0
+__device__ __forceinline__ bool is_padding(const RouteArgs &a, int t) { return a.mask && !__ldg(a.mask + t); }
+
+__device__ __forceinline__ void write_padding_route(int t, int *idx, float *gate)
+{
+    idx[2 * t] = -1;
+    idx[2 * t + 1] = -1;
+    gate[2 * t] = 0.f;
+    gate[2 * t + 1] = 0.f;
+}
+
 // The logits of token t by one block of kRouteTokenThreads threads splitting d: every
 // thread issues all its loads at once (one memory latency), then a fixed-order reduction
 // (lane tree, then the warp partials in warp order) gives the logits; thread 0 writes the
@@ -68,6 +79,10 @@ constexpr int kRouteTokenThreads = 256;
 // of u is formed in fp32, rounded to bf16, stored and used.
 __device__ __forceinline__ void route_token(const RouteArgs &a, int t)
 {
+    if (is_padding(a, t)) {   // uniform over the block
+        if (threadIdx.x == 0) write_padding_route(t, a.idx, a.gate);
+        return;
+    }
     constexpr int kWarps = kRouteTokenThreads / 32;
     __shared__ float part[kWarps][kExperts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -78,7 +78,10 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouteArgs a)
                 if (lane == j) v = acc[j][e];
             mine[e] = v;
         }
-        select_top2(mine, a.bias, t0 + lane, a.idx, a.gate);
+        if (is_padding(a, t0 + lane))
+            write_padding_route(t0 + lane, a.idx, a.gate);
+        else
+            select_top2(mine, a.bias, t0 + lane, a.idx, a.gate);
     }
 }
 

@@ -173,6 +173,71 @@ def test_tiny_residual_block(m, tiny_inputs, tiny_handle, T):
     assert err <= parity.OUT_RTOL * np.abs(dr).max() + 2 * np.abs(ref_out).max() * 2.0 ** -8, err
 
 
+def _padding_mask(T, seed):
+    g = torch.Generator().manual_seed(seed)
+    mask = (torch.rand(T, generator=g) > 0.3).to(torch.uint8)
+    mask[0], mask[-1] = 1, 0          # at least one real and one padding token
+    return mask
+
+
+@pytest.mark.parametrize("T", [8, 64, 300])
+def test_padding_mask(m, tiny_inputs, tiny_handle, T):
+    """Padding tokens (mask 0) are routed nowhere: experts -1, gates 0, no dispatched
+    route, output row 0; real tokens match the oracle as without a mask."""
+    h, layer, _ = tiny_handle
+    layer_cpu = tiny_inputs.layers[0]
+    x_cpu = tiny_inputs.x[:T]
+    mask = _padding_mask(T, 40 + T)
+    pad = mask.numpy() == 0
+    mask_dev = mask.cuda()
+    m.check(m.moe_set_padding_mask(h, mask_dev))
+    try:
+        run = parity.Run(h, x_cpu.cuda(), layer)
+    finally:
+        m.check(m.moe_set_padding_mask(h, None))
+    ref = oracle.route(x_cpu, layer_cpu["router_w"])
+    near = oracle.near_ties(ref["probs"], parity.NEAR_TIE) & ~pad
+    assert (run.idx_h[pad] == -1).all() and np.all(run.gate_h[pad] == 0.0)
+    ok = ~pad & ~near
+    assert np.array_equal(run.idx_h[ok], ref["idx"][ok])
+    np.testing.assert_allclose(run.gate_h[ok], ref["gate"][ok], rtol=parity.GATE_RTOL, atol=1e-7)
+    merged = np.where(near[:, None], run.idx_h, np.where(pad[:, None], -1, ref["idx"]))
+    counts, offsets, perm = oracle.dispatch(merged, 8)
+    assert np.array_equal(run.offsets_h, offsets)
+    assert offsets[-1] == 2 * int((~pad).sum())
+    assert np.array_equal(run.perm_h[:offsets[-1]], perm[:offsets[-1]])
+    assert torch.all(run.out_h[torch.from_numpy(pad)] == 0)
+    real = np.nonzero(~pad)[0].tolist()
+    forced = np.array([run.idx_h[t] if near[t] else (-1, -1) for t in real], dtype=np.int32)
+    out, _, _ = oracle.forward(layer_cpu, x_cpu, tokens=real, mask=mask.numpy())
+    for s_, t in enumerate(real):
+        if near[t]:
+            o, _, _ = oracle.forward(layer_cpu, x_cpu, tokens=[t], forced_idx=[forced[s_]])
+            out[s_] = o[0]
+    got = run.out_h[real].to(torch.float64).numpy()
+    assert np.abs(got - out).max() <= parity.OUT_RTOL * np.abs(out).max()
+
+
+def test_padding_mask_residual_block(m, tiny_inputs, tiny_handle):
+    """moe_block_forward leaves a padding token's residual row unchanged (bit for bit)."""
+    h, layer, _ = tiny_handle
+    T = 8
+    mask = _padding_mask(T, 77)
+    pad = torch.from_numpy(mask.numpy() == 0)
+    h_in = tiny_inputs.x[:T].clone()
+    h_dev = h_in.cuda().contiguous()
+    ones = torch.ones(256, dtype=torch.bfloat16, device="cuda")
+    m.check(m.moe_set_padding_mask(h, mask.cuda()))
+    try:
+        m.check(m.moe_block_forward(h, T, h_dev, ones, ones, 1e-5, *m.layer_args(layer)))
+        m.check(m.moe_sync_status(h))
+    finally:
+        m.check(m.moe_set_padding_mask(h, None))
+    got = h_dev.cpu()
+    assert torch.equal(got[pad], h_in[pad])
+    assert not torch.equal(got[~pad], h_in[~pad])
+
+
 def test_pack_weight_is_a_transpose(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
