@@ -54,15 +54,17 @@ struct CfgTS {
     static constexpr int CH = (kBKT / 16) / KP;             // 16-byte chunks per converter thread and stage
     static constexpr int STG = NB * kBM * kBKT;             // int8 staging bytes per stage
     static constexpr int BBYTES = BN * KSTAGE * 2;          // bf16 activation bytes per stage
-    static constexpr int NDB = (UP && BN == 128) ? 1 : 2;   // accumulator buffers in TMEM
-    // Two MMA issuers, one per box of a stage, each into an accumulator of its own: the
+    // Two MMA issuers, each into an accumulator of its own: per box of a stage for the
     // up-projection (one accumulator per matrix anyway) and the narrow down-projection (one per
-    // k-box, summed by the epilogue).  The converter warps keep every SM sub-partition's issue
-    // slots busy, and a single issuing thread, which spends several instructions per MMA, then
-    // falls behind the tensor core at the small N of decode-sized tiles.
-    static constexpr bool DUAL = UP || (K2 && BN <= 32);
+    // k-box); per half of the stage's 8 K slices for the 128-route down-projection, whose stage
+    // holds one box (KSPLIT).  The epilogue sums a down-projection's two accumulators.  The
+    // converter warps keep every SM sub-partition's issue slots busy, and a single issuing
+    // thread, which spends several instructions per MMA, then falls behind the tensor core.
+    static constexpr bool KSPLIT = !UP && !K2;
+    static constexpr bool DUAL = UP || (K2 && BN <= 32) || KSPLIT;
     static constexpr int NACC = DUAL ? 2 : 1;               // accumulators per tile
     static constexpr int ACC = NACC * BN;                   // TMEM columns of one accumulator buffer
+    static constexpr int NDB = (NACC * BN > 128) ? 1 : 2;   // accumulator buffers in TMEM
     static constexpr int A_COLS = NB * kBKT / 2;            // TMEM columns of one A stage
     static constexpr int S2 = cmin(4, (512 - NDB * ACC) / A_COLS);   // A (TMEM) + B (smem) ring
     static constexpr int S1 = cmin(12, (kSmemBudget - S2 * BBYTES) / STG);   // int8 staging ring
@@ -333,19 +335,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
 #pragma unroll
                     for (int bx = 0; bx < C::NB; ++bx) {
-                        if (C::DUAL && bx != mine) continue;
 #pragma unroll
                         for (int kk = 0; kk < kBKT / 16; ++kk) {
+                            // issuer / accumulator of this MMA: the box, or the half of the K slices
+                            const int who = C::KSPLIT ? (kk >> 2) : bx;
+                            if (C::DUAL && who != mine) continue;
                             // K slice of the stage's activation tile; both matrices of the
                             // up-projection use the same slices, the k-boxes of the down-projection
                             // consecutive ones
                             const int kg = (UP ? 0 : bx * (kBKT / 16)) + kk;
                             const uint64_t bdesc =
                                 desc_sw128(bbase + (kg >> 2) * (BN * 128) + (kg & 3) * 32, 16, 1024);
-                            // the item's first stage starts its accumulator
+                            // the item's first MMA into an accumulator starts it
                             const int kr = ks - wi.k0;
-                            const uint32_t acc = C::DUAL ? ((kr | kk) != 0) : ((kr | bx | kk) != 0);
-                            umma_bf16_ts(dcol + (C::DUAL ? bx : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc,
+                            const int kf = C::KSPLIT ? (kk & 3) : kk;
+                            const uint32_t acc = C::DUAL ? ((kr | kf) != 0) : ((kr | bx | kk) != 0);
+                            umma_bf16_ts(dcol + (C::DUAL ? who : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc,
                                          idesc, acc);
                         }
                     }
