@@ -94,6 +94,19 @@ def draw_layer(d: int, F: int, E: int, g: torch.Generator, device) -> Dict[str, 
     return dict(router_w=router_w, wl=wl, sl=sl, wv=wv, sv=sv, w1=w1, s1=s1)
 
 
+def block_scales(layer: Dict[str, torch.Tensor], kb: int, g: torch.Generator) -> Dict[str, torch.Tensor]:
+    """The layer with per-block scales instead of per-output-channel ones: every block of kb
+    input rows of every matrix gets its own scale row ([E, in/kb, out]), drawn like the
+    per-channel scales.  Weights and router are shared with ``layer``."""
+    E, d, F = layer["wl"].shape
+    dev = layer["wl"].device
+    out = dict(layer)
+    out["sl"] = _scale((E, d // kb, F), d, g, dev)
+    out["sv"] = _scale((E, d // kb, F), d, g, dev)
+    out["s1"] = _scale((E, F // kb, d), d, g, dev)
+    return out
+
+
 def draw_tokens(T: int, d: int, g: torch.Generator, device) -> torch.Tensor:
     return torch.randn((T, d), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
 

@@ -72,9 +72,9 @@ def lib():
         L.moe_oracle_dispatch.restype = i
         L.moe_oracle_dispatch.argtypes = [i, i, P, P, P, P]
         L.moe_oracle_expert_ffn.restype = i
-        L.moe_oracle_expert_ffn.argtypes = [i, i, P, P, P, P, P, P, P, P, P, i, i]
+        L.moe_oracle_expert_ffn.argtypes = [i, i, P, P, P, P, P, P, P, P, P, i, i, i]
         L.moe_oracle_forward.restype = i
-        L.moe_oracle_forward.argtypes = [i, i, i, i, P, P, P, P, P, P, P, P, P, P, i, P, P, P, P, P, i, i]
+        L.moe_oracle_forward.argtypes = [i, i, i, i, P, P, P, P, P, P, P, P, P, P, i, P, P, P, P, P, i, i, i]
         L.moe_oracle_rmsnorm.restype = i
         L.moe_oracle_rmsnorm.argtypes = [i, i, P, P, ctypes.c_double, P]
         _lib = L
@@ -178,6 +178,13 @@ def dispatch(idx, E: int):
     return counts, offsets, perm
 
 
+def scale_block(layer) -> int:
+    """Block of inputs sharing a scale: 0 when the scales are per output channel ([E, out]),
+    else in / (number of scale rows) for per-block scales ([E, in/kb, out])."""
+    sl, wl = layer["sl"], layer["wl"]
+    return 0 if len(sl.shape) == 2 else wl.shape[1] // sl.shape[1]
+
+
 def expert_ffn(xt: np.ndarray, layer, e: int, nthreads: int = 0, gelu_kind: int = 0,
                return_h: bool = False):
     """One expert's gated-GELU FFN on one fp64 token row."""
@@ -188,8 +195,9 @@ def expert_ffn(xt: np.ndarray, layer, e: int, nthreads: int = 0, gelu_kind: int 
     E, d, F = wl.shape
     y = np.zeros(d, np.float64)
     h = np.zeros(F, np.float64)
-    _check(lib().moe_oracle_expert_ffn(d, F, _p(xt), _p(wl[e]), _p(sl[e]), _p(wv[e]), _p(sv[e]),
-                                       _p(w1[e]), _p(s1[e]), _p(h), _p(y), nthreads, gelu_kind),
+    _check(lib().moe_oracle_expert_ffn(d, F, _p(xt), _p(wl[e]), _p(np.ascontiguousarray(sl[e])), _p(wv[e]),
+                                       _p(np.ascontiguousarray(sv[e])), _p(w1[e]), _p(np.ascontiguousarray(s1[e])),
+                                       _p(h), _p(y), nthreads, gelu_kind, scale_block(layer)),
            "expert_ffn")
     return (y, h) if return_h else y
 
@@ -221,7 +229,7 @@ def forward(layer, x, bias=None, tokens: Optional[Sequence[int]] = None, forced_
     gate = np.zeros((n, 2), np.float64)
     _check(lib().moe_oracle_forward(T, d, F, E, _p(xb), _p(rw), _p(b), _p(wl), _p(sl), _p(wv),
                                     _p(sv), _p(w1), _p(s1), _p(tk), n, _p(fi), _p(mk), _p(out), _p(idx),
-                                    _p(gate), nthreads, gelu_kind), "forward")
+                                    _p(gate), nthreads, gelu_kind, scale_block(layer)), "forward")
     return out, idx, gate
 
 

@@ -214,7 +214,9 @@ typedef struct {
     int d, F, gelu_kind;
     const double *xt;                 /* [d] token, fp64                      */
     const int8_t *wl, *wv, *w1;       /* [d,F], [d,F], [F,d] int8 of expert e */
-    const uint16_t *sl, *sv, *s1;     /* [F], [F], [d] bf16 scales            */
+    const uint16_t *sl, *sv, *s1;     /* bf16 scales: [F], [F], [d] per output channel, or
+                                         [d/kb,F], [d/kb,F], [F/kb,d] per block of kb inputs */
+    int kb;                           /* scale block along the input dimension; 0: none */
     double *h;                        /* [F] gelu(linear) * linear_v           */
     double *y;                        /* [d] linear_1(h)                      */
     int lo, hi;                       /* this worker's output column range     */
@@ -223,6 +225,8 @@ typedef struct {
 /* linear and linear_v over output columns f in [lo, hi):
  *   a[f] = sum_i x[i] * (Wl[i,f] * sl[f]),  v[f] = sum_i x[i] * (Wv[i,f] * sv[f])
  *   h[f] = gelu(a[f]) * v[f]
+ * (with block scales, sl[i / kb, f] and sv[i / kb, f]: "Grok-1 Admin & Architecture
+ * Guide", section 3 "Quantized weights", per-block dequant scales).
  * The dequantised weight Wl[i,f]*sl[f] is formed first (exact in fp64: an
  * 8-bit integer times an 8-bit-significand scale), then the dot product. */
 static void *ffn_up_worker(void *arg)
@@ -235,11 +239,14 @@ static void *ffn_up_worker(void *arg)
     double *restrict s_l = malloc((size_t)n * sizeof(double));
     double *restrict s_v = malloc((size_t)n * sizeof(double));
     if (!a || !v || !s_l || !s_v) { free(a); free(v); free(s_l); free(s_v); return (void *)1; }
-    for (int f = 0; f < n; ++f) {
-        s_l[f] = bf16_to_f64(j->sl[j->lo + f]);
-        s_v[f] = bf16_to_f64(j->sv[j->lo + f]);
-    }
     for (int i = 0; i < j->d; ++i) {
+        if (i == 0 || (j->kb && i % j->kb == 0)) {   /* the scale row of this input */
+            const size_t row = j->kb ? (size_t)(i / j->kb) * j->F : 0;
+            for (int f = 0; f < n; ++f) {
+                s_l[f] = bf16_to_f64(j->sl[row + j->lo + f]);
+                s_v[f] = bf16_to_f64(j->sv[row + j->lo + f]);
+            }
+        }
         const double xi = j->xt[i];
         const int8_t *restrict rl = j->wl + (size_t)i * j->F + j->lo;
         const int8_t *restrict rv = j->wv + (size_t)i * j->F + j->lo;
@@ -256,7 +263,8 @@ static void *ffn_up_worker(void *arg)
     return NULL;
 }
 
-/* linear_1 over output columns c in [lo, hi):  y[c] = sum_f h[f] * (W1[f,c] * s1[c]) */
+/* linear_1 over output columns c in [lo, hi):  y[c] = sum_f h[f] * (W1[f,c] * s1[c])
+ * (with block scales, s1[f / kb, c]) */
 static void *ffn_down_worker(void *arg)
 {
     ffn_job *j = arg;
@@ -265,8 +273,11 @@ static void *ffn_down_worker(void *arg)
     double *restrict acc = calloc((size_t)n, sizeof(double));
     double *restrict s = malloc((size_t)n * sizeof(double));
     if (!acc || !s) { free(acc); free(s); return (void *)1; }
-    for (int c = 0; c < n; ++c) s[c] = bf16_to_f64(j->s1[j->lo + c]);
     for (int f = 0; f < j->F; ++f) {
+        if (f == 0 || (j->kb && f % j->kb == 0)) {
+            const size_t row = j->kb ? (size_t)(f / j->kb) * j->d : 0;
+            for (int c = 0; c < n; ++c) s[c] = bf16_to_f64(j->s1[row + j->lo + c]);
+        }
         const double hf = j->h[f];
         const int8_t *restrict r = j->w1 + (size_t)f * j->d + j->lo;
         for (int c = 0; c < n; ++c) acc[c] += hf * ((double)r[c] * s[c]);
@@ -310,18 +321,20 @@ static int run_split(void *(*fn)(void *), ffn_job *base, int ncols, int nthreads
 
 /*
  * One expert e on one token: y = linear_1( gelu(linear(x)) * linear_v(x) ).
- * xt fp64 [d]; wl, wv int8 [d,F]; w1 int8 [F,d]; sl, sv bf16 [F]; s1 bf16 [d]
- * (already offset to expert e); y fp64 [d].  h (fp64 [F]) may be NULL.
+ * xt fp64 [d]; wl, wv int8 [d,F]; w1 int8 [F,d]; scales bf16, per output channel
+ * (kb = 0: sl, sv [F], s1 [d]) or per block of kb inputs (sl, sv [d/kb,F], s1 [F/kb,d]),
+ * all already offset to expert e; y fp64 [d].  h (fp64 [F]) may be NULL.
  */
 ORACLE_API int moe_oracle_expert_ffn(int d, int F, const double *xt, const int8_t *wl,
                                      const uint16_t *sl, const int8_t *wv, const uint16_t *sv,
                                      const int8_t *w1, const uint16_t *s1, double *h_out,
-                                     double *y, int nthreads, int gelu_kind)
+                                     double *y, int nthreads, int gelu_kind, int kb)
 {
     if (d <= 0 || F <= 0 || !xt || !wl || !sl || !wv || !sv || !w1 || !s1 || !y) return OR_EINVAL;
+    if (kb < 0 || (kb && (d % kb || F % kb))) return OR_EINVAL;
     double *h = h_out ? h_out : malloc((size_t)F * sizeof(double));
     if (!h) return OR_ENOMEM;
-    ffn_job base = {d, F, gelu_kind, xt, wl, wv, w1, sl, sv, s1, h, y, 0, 0};
+    ffn_job base = {d, F, gelu_kind, xt, wl, wv, w1, sl, sv, s1, kb, h, y, 0, 0};
     nthreads = default_threads(nthreads);
     int rc = run_split(ffn_up_worker, &base, F, nthreads);
     if (rc == OR_OK) rc = run_split(ffn_down_worker, &base, d, nthreads);
@@ -338,6 +351,8 @@ ORACLE_API int moe_oracle_expert_ffn(int d, int F, const double *xt, const int8_
  * forced_idx (int32 [n_sel,2], may be NULL) names the two experts to use; the
  * gates are then those experts' softmax probabilities.
  * Weights: wl, wv int8 [E,d,F], w1 int8 [E,F,d]; sl, sv bf16 [E,F]; s1 bf16 [E,d].
+ * kb: scale block along the input dimension (0: one scale per output channel), as
+ * in moe_oracle_expert_ffn.
  * mask (uint8 [T], may be NULL = every token real): a token t with mask[t] == 0 is
  * padding, the padding_mask of the MoE call in the grok-field-guide source-code map,
  * fourth stop (moe(rms_norm(h), padding_mask)); it is routed nowhere: out row 0,
@@ -349,7 +364,7 @@ ORACLE_API int moe_oracle_forward(int T, int d, int F, int E, const uint16_t *x,
                                   const uint16_t *sl, const int8_t *wv, const uint16_t *sv,
                                   const int8_t *w1, const uint16_t *s1, const int32_t *tokens,
                                   int n_sel, const int32_t *forced_idx, const uint8_t *mask, double *out,
-                                  int32_t *idx, double *gate, int nthreads, int gelu_kind)
+                                  int32_t *idx, double *gate, int nthreads, int gelu_kind, int kb)
 {
     if (T < 0 || d <= 0 || F <= 0 || E < 2 || E > 64 || !x || !router_w || !wl || !sl || !wv ||
         !sv || !w1 || !s1 || !out)
@@ -383,10 +398,13 @@ ORACLE_API int moe_oracle_forward(int T, int d, int F, int E, const uint16_t *x,
         for (int i = 0; i < d; ++i) o[i] = 0.0;
         for (int j = 0; j < 2 && rc == OR_OK; ++j) {
             int e = sel[j];
-            rc = moe_oracle_expert_ffn(d, F, xt, wl + (size_t)e * d * F, sl + (size_t)e * F,
-                                       wv + (size_t)e * d * F, sv + (size_t)e * F,
-                                       w1 + (size_t)e * F * d, s1 + (size_t)e * d, NULL, y,
-                                       nthreads, gelu_kind);
+            /* per expert: F (or d/kb * F) scales of linear / linear_v, d (or F/kb * d) of linear_1 */
+            const size_t up_s = kb ? (size_t)(d / kb) * F : (size_t)F;
+            const size_t dn_s = kb ? (size_t)(F / kb) * d : (size_t)d;
+            rc = moe_oracle_expert_ffn(d, F, xt, wl + (size_t)e * d * F, sl + (size_t)e * up_s,
+                                       wv + (size_t)e * d * F, sv + (size_t)e * up_s,
+                                       w1 + (size_t)e * F * d, s1 + (size_t)e * dn_s, NULL, y,
+                                       nthreads, gelu_kind, kb);
             /* combine in route order: slot 0 first, then slot 1 */
             for (int i = 0; i < d; ++i) o[i] += probs[e] * y[i];
         }

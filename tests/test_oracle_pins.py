@@ -289,6 +289,37 @@ def test_padding_mask_routes_nothing(tiny):
     assert np.array_equal(blk["h_out"][~mask[:16]], blk["h_in"][~mask[:16]])
 
 
+def test_block_scales_match_numpy(tiny):
+    """Per-block scales ([E, in/kb, out]): the oracle's expert FFN equals numpy float64
+    matmuls on weights dequantised with np.repeat of the scale rows over their blocks."""
+    layer = moe_synth.block_scales(tiny.layers[0], 128, torch.Generator().manual_seed(21))
+    assert oracle.scale_block(layer) == 128
+    f = lambda t: t.to(torch.float64).numpy()
+    rep = lambda sc, n: np.repeat(f(sc), n, axis=1)        # [E, in/kb, out] -> [E, in, out]
+    Wl = f(layer["wl"]) * rep(layer["sl"], 128)
+    Wv = f(layer["wv"]) * rep(layer["sv"], 128)
+    W1 = f(layer["w1"]) * rep(layer["s1"], 128)
+    x64 = tiny.x[:3].to(torch.float64).numpy()
+    for e in (0, 5):
+        for t in range(3):
+            y = oracle.expert_ffn(x64[t], layer, e, gelu_kind=1)
+            ref = (_erf_gelu(x64[t] @ Wl[e]) * (x64[t] @ Wv[e])) @ W1[e]
+            np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12 * np.abs(ref).max())
+
+
+def test_block_scales_equal_rows_reduce_to_channel_scales(tiny):
+    """Block scales whose rows are all the per-channel scale give the per-channel layer bit for bit."""
+    layer = tiny.layers[0]
+    E, d, F = layer["wl"].shape
+    blk = dict(layer)
+    blk["sl"] = layer["sl"][:, None, :].expand(E, d // 128, F).contiguous()
+    blk["sv"] = layer["sv"][:, None, :].expand(E, d // 128, F).contiguous()
+    blk["s1"] = layer["s1"][:, None, :].expand(E, F // 128, d).contiguous()
+    out, idx, _ = oracle.forward(layer, tiny.x[:16])
+    out_b, idx_b, _ = oracle.forward(blk, tiny.x[:16])
+    assert np.array_equal(out, out_b) and np.array_equal(idx, idx_b)
+
+
 def test_linear_in_output_scale(tiny):
     layer = dict(tiny.layers[0])
     out, _, _ = oracle.forward(layer, tiny.x, tokens=[0, 1, 2])
