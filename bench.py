@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--tokens", type=int, default=None, help="override T")
     p.add_argument("--ffn", type=int, default=None, help="override the FFN width")
     p.add_argument("--skip-extras", action="store_true", help="skip the per-kernel and end-to-end passes")
+    p.add_argument("--scale-block", type=int, choices=(0, 128), default=0,
+                   help="weight scale format: 0 per output channel, 128 per block of 128 inputs (packed layout)")
     p.add_argument("--layout", choices=("packed", "in_out"), default="packed",
                    help="weight layout: packed = tiles written once at load (TMEM path); in_out = as drawn")
     return p.parse_args()
@@ -206,12 +208,15 @@ def recorded_traffic(workload, kernel):
     return ent.get("bytes_per_launch")
 
 
-def algorithmic_work(w, T, n_touched, counts):
-    """Per-launch algorithmic bytes and FLOPs of the up- and down-projection kernels."""
+def algorithmic_work(w, T, n_touched, counts, kblock=0):
+    """Per-launch algorithmic bytes and FLOPs of the up- and down-projection kernels
+    (kblock: 0 = one bf16 scale per output channel, else one per block of kblock inputs)."""
     d, F = w.d, w.F
     R = 2 * T
-    up_bytes = n_touched * (2 * d * F + 2 * 2 * F) + R * d * 2 + R * F * 2
-    dn_bytes = n_touched * (F * d + 2 * d) + R * F * 2 + R * d * 4
+    up_scales = 2 * 2 * F * (d // kblock if kblock else 1)
+    dn_scales = 2 * d * (F // kblock if kblock else 1)
+    up_bytes = n_touched * (2 * d * F + up_scales) + R * d * 2 + R * F * 2
+    dn_bytes = n_touched * (F * d + dn_scales) + R * F * 2 + R * d * 4
     up_flops = 2.0 * R * d * F * 2
     dn_flops = 2.0 * R * F * d
     return dict(up_bytes=up_bytes, dn_bytes=dn_bytes, up_flops=up_flops, dn_flops=dn_flops)
@@ -237,11 +242,15 @@ def run_native(args, world, rank, local):
         inp.x = moe_synth.draw_tokens(w.T, w.d, g, dev)
     T = w.T
     layers = inp.layers
+    if args.scale_block:   # per-block scale format: the same weights, one scale row per 128 inputs
+        gs = moe_synth.generator(w.seed + 2000, dev)
+        layers = [moe_synth.block_scales(l, args.scale_block, gs) for l in layers]
     bias = inp.bias
     stream = torch.cuda.current_stream(dev)
 
     h = moe.MoELayer(w.d, w.F, w.E, w.k)
     moe.check(moe.moe_set_router_bias(h.h, bias))
+    moe.check(moe.moe_set_scale_block(h.h, args.scale_block))
     if args.layout == "packed":
         # one-time weight-load step, outside every timed region: K-major int8 copies
         moe.check(moe.moe_set_weight_layout(h.h, moe.MOE_LAYOUT_PACKED))
@@ -341,7 +350,7 @@ def run_native(args, world, rank, local):
                "d2h_bytes_per_step": nb, "ms_per_step": e2e_ms, "api": "moe_forward_host"}
 
     peaks, peak_src = measured_peaks()
-    work = algorithmic_work(w, T, n_touched, counts)
+    work = algorithmic_work(w, T, n_touched, counts, args.scale_block)
     up_ms = per_launch["up_proj"]
     dn_ms = per_launch["down_proj"]
     if args.workload in ("prefill", "skewed"):
@@ -377,7 +386,9 @@ def run_native(args, world, rank, local):
         "dtype": "bf16", "data": "synthetic (seeded; random-init int8 weights of the Grok-1 MoE shape)",
         "config": {"workload": args.workload, "T_per_gpu": T, "d_model": w.d, "ffn": w.F, "experts": w.E,
                    "top_k": w.k, "blocks": w.blocks or 1,
-                   "weights": "int8 + bf16 per-output-channel scales, layout " + args.layout +
+                   "weights": "int8 + bf16 " + ("scales per block of %d inputs" % args.scale_block
+                                                if args.scale_block else "per-output-channel scales") +
+                              ", layout " + args.layout +
                               (" (packed once at load, untimed)" if args.layout == "packed" else ""),
                    "l2": "inputs larger than L2 (%.2f GB of weights per step)" % (layer_bytes / 1e9),
                    "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],

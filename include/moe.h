@@ -116,6 +116,21 @@ MOE_API int moe_set_router_bias(moe_handle h, const float *bias);
 MOE_API int moe_set_padding_mask(moe_handle h, const uint8_t *mask);
 
 /*
+ * Scale format of the int8 weights: "Grok-1 Admin & Architecture Guide", section 3
+ * "Quantized weights", stores each weight as int8 values with per-block dequant
+ * scales (w.weight * w.scales).  kb = 0 (the default): one bf16 scale per output
+ * channel, s_lin, s_v [E, ffn] and s_1 [E, d].  kb = 128: one bf16 scale per output
+ * channel and block of 128 consecutive input rows, s_lin, s_v [E, d/128, ffn] and
+ * s_1 [E, ffn/128, d]; the weight at input row i uses scale row i / 128.  With
+ * block scales each weight is dequantised to bf16(w * s) (one rounding) before the
+ * MMA; per-channel scales are applied to the fp32 sums instead.  Applies to later
+ * forwards; block scales need MOE_LAYOUT_PACKED (forwards otherwise return
+ * MOE_EUNSUPPORTED).  Errors: MOE_EINVAL for a NULL handle or d / ffn not
+ * multiples of kb; MOE_EUNSUPPORTED for any other kb.
+ */
+MOE_API int moe_set_scale_block(moe_handle h, int kb);
+
+/*
  * The MoE layer on T tokens ("Mixture of Experts (MoELayer + Router)", steps 1-4).
  *   x    bf16 [T, d]   input tokens
  *   out  bf16 [T, d]   output; must not overlap x or the weights

@@ -36,6 +36,7 @@ KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine
 # every symbol include/moe.h declares
 EXPORTS = (
     "moe_strerror", "moe_version", "moe_create", "moe_destroy", "moe_set_router_bias", "moe_set_padding_mask",
+    "moe_set_scale_block",
     "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing",
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
     "moe_set_weight_layout", "moe_pack_weight", "moe_route_noalloc",
@@ -62,6 +63,7 @@ def _load() -> ctypes.CDLL:
         "moe_destroy": (I, [P]),
         "moe_set_router_bias": (I, [P, P]),
         "moe_set_padding_mask": (I, [P, P]),
+        "moe_set_scale_block": (I, [P, I]),
         "moe_forward": (I, [P, I, P, P, P, P, P, P, P, P, P, P]),
         "moe_forward_host": (I, [P, I, P, P, P, P, P, P, P, P, P, P]),
         "moe_block_forward": (I, [P, I, P, P, P, F, P, P, P, P, P, P, P, P]),
@@ -139,6 +141,11 @@ def moe_set_router_bias(h, bias) -> int:
 def moe_set_padding_mask(h, mask) -> int:
     """mask: device uint8 [T] (0 = padding token) or None; kept, not copied."""
     return _lib.moe_set_padding_mask(h, _ptr(mask))
+
+
+def moe_set_scale_block(h, kb: int) -> int:
+    """0: per-output-channel scales; 128: per block of 128 input rows ([E, in/128, out])."""
+    return _lib.moe_set_scale_block(h, int(kb))
 
 
 def moe_forward(h, T, x, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, out, stream=None) -> int:

@@ -399,8 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = m * kBM + q * 32 + lane;
             const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::ACC;
             const int row0 = poff[e] + n * BN;
-            const float sc0 = __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
-            const float sc1 = UP ? __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]) : 0.f;
+            // per-channel scales here; the per-block format applied them while dequantising
+            const float sc0 = a.kblock ? 1.f : __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
+            const float sc1 = !UP ? 0.f : a.kblock ? 1.f : __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
             const bool whole = wi.piece < 0;   // uniform over the CTA
             if (!whole) {
                 // a piece: its partial sums go to the workspace, [piece][row][accumulator column]
@@ -481,6 +482,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         PS_VAR(c_ctail);
         for (int item = blockIdx.x; item < wl.items; item += gridDim.x) {
             const WorkItem wi = work_item(wl, item, a.ksteps);
+            // per-block scale format: this thread's feature row in the scale rows of its box;
+            // the scale row of a stage is its first reduction row / kScaleBlock
+            const __nv_bfloat16 *srow = nullptr;
+            if (a.kblock) {
+                int e, m, n, s;
+                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                const int k0 = s * a.ksteps * C::KSTAGE + (UP ? 0 : box * kBKT);
+                srow = ((UP && box == 1) ? a.s1 : a.s0) +
+                       (static_cast<size_t>(e) * (a.K / kScaleBlock) + k0 / kScaleBlock) * a.M + m * kBM + fr;
+            }
             bool ok = true;
             for (int ks = wi.k0; ks < wi.k1; ++ks) {
                 PS_NOW(t0);
@@ -493,6 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint4 v[C::CH];
 #pragma unroll
                 for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
+                __nv_bfloat162 sc2;   // this row's block scale (per-block format)
+                if (a.kblock) {
+                    const __nv_bfloat16 sv = srow[static_cast<size_t>(ks) * (C::KSTAGE / kScaleBlock) * a.M];
+                    sc2 = __halves2bfloat162(sv, sv);
+                }
                 const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + box * (kBKT / 2) + j0 * 8;
                 __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
                 // each 16-byte chunk (16 reduction elements = 8 TMEM columns) is stored as soon
@@ -508,6 +524,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     words[5] = i8x2_to_bf16x2(v[c].z, 0x4342);
                     words[6] = i8x2_to_bf16x2(v[c].w, 0x4140);
                     words[7] = i8x2_to_bf16x2(v[c].w, 0x4342);
+                    if (a.kblock) {   // dequantised weight bf16(w * s): exact w, one rounding of the product
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            __nv_bfloat162 wq = *reinterpret_cast<const __nv_bfloat162 *>(&words[q]);
+                            wq = __hmul2(wq, sc2);
+                            words[q] = *reinterpret_cast<const uint32_t *>(&wq);
+                        }
+                    }
                     tmem_st8(taddr + c * 8, words);
                 }
                 PS_ADD(c_cwork, t1);

@@ -9,6 +9,7 @@
 namespace moe {
 
 constexpr int kExperts = 8;       // E supported by the router kernel
+constexpr int kScaleBlock = 128;   // reduction rows sharing a scale in the per-block scale format
 constexpr int kTopK = 2;          // picks per token
 constexpr int kBM = 128;          // output features per GEMM tile (TMEM lanes)
 constexpr int kBK = 64;           // reduction elements per pipeline stage (128 B of bf16)
@@ -69,6 +70,10 @@ struct GemmArgs {
     float *slots;               // DOWN output [splits, T, 2, M]
     int *err;                   // device error word
     long long timeout_ns;
+    // scale format: 0 = one scale per output channel, s0/s1 [E, M] (applied in the epilogue);
+    // kScaleBlock = per block of kScaleBlock reduction rows, s0/s1 [E, K / kScaleBlock, M]
+    // (applied while dequantising, TMEM-operand kernels only)
+    int kblock;
     // last-wave pieces (TMEM-operand kernels): partial accumulators and per-tile tickets
     float *part;                // [gridDim.x, 128, accumulator columns] fp32, or nullptr: no pieces
     unsigned int *tickets;      // [gridDim.x], zero, left zero by every launch that completes

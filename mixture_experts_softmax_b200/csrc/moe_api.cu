@@ -65,6 +65,7 @@ struct moe_ctx {
 
     const float *bias = nullptr;
     const uint8_t *mask = nullptr;   // padding mask of the next forwards (device, >= T bytes)
+    int kblock = 0;                  // scale format: 0 per output channel, kScaleBlock per block
     long long timeout_ns = 2000000000LL;
     int layout = MOE_LAYOUT_IN_OUT;
 
@@ -362,6 +363,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     int *rperm = static_cast<int *>(h->b_rperm.ptr);
 
     const bool ts = h->layout == MOE_LAYOUT_PACKED;
+    if (h->kblock && !ts) return MOE_EUNSUPPORTED;   // block scales: TMEM-operand kernels only
     const CUtensorMap *m_wl, *m_wv, *m_w1, *m_xp, *m_h;
     if ((rc = weight_map(h, w_lin, 0, &m_wl)) != MOE_OK) return rc;
     if ((rc = weight_map(h, w_v, 0, &m_wv)) != MOE_OK) return rc;
@@ -413,6 +415,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.h = static_cast<__nv_bfloat16 *>(h->b_h.ptr);
     up.err = h->err;
     up.timeout_ns = h->timeout_ns;
+    up.kblock = h->kblock;
     if (ts) {
         up.part = static_cast<float *>(h->b_part.ptr);
         up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
@@ -526,6 +529,15 @@ MOE_API int moe_set_padding_mask(moe_handle h, const uint8_t *mask)
 {
     if (!h) return MOE_EINVAL;
     h->mask = mask;
+    return MOE_OK;
+}
+
+MOE_API int moe_set_scale_block(moe_handle h, int kb)
+{
+    if (!h) return MOE_EINVAL;
+    if (kb != 0 && kb != kScaleBlock) return MOE_EUNSUPPORTED;
+    if (kb && (h->d % kb || h->F % kb)) return MOE_EINVAL;
+    h->kblock = kb;
     return MOE_OK;
 }
 

@@ -238,6 +238,28 @@ def test_padding_mask_residual_block(m, tiny_inputs, tiny_handle):
     assert not torch.equal(got[~pad], h_in[~pad])
 
 
+@pytest.mark.parametrize("T", [8, 64, 300])
+def test_block_scales(m, tiny_inputs, tiny_handle, T):
+    """Per-block weight scales (one per 128 input rows and output channel): the packed layout
+    dequantises bf16(w * s) before the MMA and matches the oracle; the API layout refuses."""
+    h, _, layout = tiny_handle
+    layer_cpu = moe_synth.block_scales(tiny_inputs.layers[0], 128, torch.Generator().manual_seed(33))
+    dev = parity.to_dev(layer_cpu)
+    x_cpu = tiny_inputs.x[:T]
+    m.check(m.moe_set_scale_block(h, 128))
+    try:
+        if layout != m.MOE_LAYOUT_PACKED:
+            out = torch.empty((T, 256), dtype=torch.bfloat16, device="cuda")
+            assert m.moe_forward(h, T, x_cpu.cuda(), *m.layer_args(dev), out) == m.MOE_EUNSUPPORTED
+            return
+        run = parity.Run(h, x_cpu.cuda(), m.pack_layer(h, dev))
+    finally:
+        m.check(m.moe_set_scale_block(h, 0))
+    ref = oracle.route(x_cpu, layer_cpu["router_w"])
+    near = parity.check_routing(run, ref, 8)
+    parity.check_output(run, layer_cpu, x_cpu, range(T), near)
+
+
 def test_pack_weight_is_a_transpose(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
