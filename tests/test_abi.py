@@ -104,6 +104,22 @@ def test_forward_argument_checks_on_host(m):
         m.moe_destroy(h)
 
 
+def test_setter_argument_checks(m):
+    """Handle settings are validated on the host; they need no GPU."""
+    rc, h = m.moe_create(256, 512, 8, 2)
+    assert rc == 0
+    try:
+        assert m.moe_set_scale_block(None, 0) == m.MOE_EINVAL
+        assert m.moe_set_scale_block(h, 64) == m.MOE_EUNSUPPORTED
+        assert m.moe_set_scale_block(h, 128) == m.MOE_OK
+        assert m.moe_set_scale_block(h, 0) == m.MOE_OK
+        assert m.moe_set_padding_mask(None, None) == m.MOE_EINVAL
+        assert m.moe_set_padding_mask(h, (1 << 20) + 3) == m.MOE_OK     # kept, not dereferenced here
+        assert m.moe_set_padding_mask(h, None) == m.MOE_OK
+    finally:
+        m.moe_destroy(h)
+
+
 def test_forward_without_gpu_reports_no_device(m):
     import torch
     if torch.cuda.is_available():
