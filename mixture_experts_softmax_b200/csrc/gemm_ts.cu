@@ -76,7 +76,7 @@ struct CfgTS {
     // barriers: stg_full[S1] stg_empty[S1] a_full[S2] b_full[S2] op_empty[S2] acc_full[NDB] acc_empty[NDB] drain[2]
     static constexpr int NBAR = 2 * S1 + 3 * S2 + 2 * NDB + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int MISC_BYTES = 16 + 2 * 4 * 40;
+    static constexpr int MISC_BYTES = 16 + 3 * 4 * 40;   // tmem addr, flags, prefix[40], poff[40], roff[40]
     static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;
     static_assert(S1 >= 2 && S2 >= 2, "rings too shallow");
     static_assert(SMEM <= 227 * 1024, "shared memory over the per-CTA limit");
@@ -97,7 +97,7 @@ __device__ __forceinline__ constexpr uint32_t idesc_ts()
 // from the full-K sums x0 (and x1: the second matrix, or the second k-box):
 //   up-projection:   H[r, f] = bf16( gelu(s0 * x0) * (s1 * x1) )
 //   down-projection: slot[s, t, j, f] = gate[t, j] * s0 * (x0 + x1)   (k-box sums in this order)
-// rows r = row0 + c + i whose route id is -1 (padding) are skipped.
+// padding rows (route id -1; for the up-projection: tile rows from nreal on) are skipped.
 struct EpiOut {
     const int *rperm;
     const float *gate;
@@ -107,14 +107,15 @@ struct EpiOut {
 };
 
 template <bool UP, int NACC>
-__device__ __forceinline__ void epilogue_chunk(const EpiOut &a, int row0, int c, int f, int s, float sc0, float sc1,
-                                               const float (&x0)[16], const float (&x1)[16])
+__device__ __forceinline__ void epilogue_chunk(const EpiOut &a, int row0, int nreal, int c, int f, int s, float sc0,
+                                               float sc1, const float (&x0)[16], const float (&x1)[16])
 {
     if constexpr (UP) {
+        // the tile's real rows are its first nreal rows (the rest pad the expert's segment)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int r = row0 + c + i;
-            if (__ldg(a.rperm + r) >= 0)
+            if (c + i < nreal)
                 a.h[static_cast<size_t>(r) * a.M + f] = __float2bfloat16_rn(gelu_tanh(sc0 * x0[i]) * (sc1 * x1[i]));
         }
     } else {
@@ -137,8 +138,8 @@ __device__ __forceinline__ void epilogue_chunk(const EpiOut &a, int row0, int c,
 // of line: it runs at most once per split tile and would otherwise raise the register
 // pressure of the whole kernel.
 template <bool UP, int BN, int NACC, int ACC>
-__device__ __noinline__ void finish_pieces(const EpiOut a, const float *p0, int P, int c0, int c1, int row0, int f,
-                                           int s, float sc0, float sc1)
+__device__ __noinline__ void finish_pieces(const EpiOut a, const float *p0, int P, int c0, int c1, int row0,
+                                           int nreal, int f, int s, float sc0, float sc1)
 {
     const size_t pstride = static_cast<size_t>(kBM) * ACC;
     for (int c = c0; c < c1; c += 16) {
@@ -161,7 +162,7 @@ __device__ __noinline__ void finish_pieces(const EpiOut a, const float *p0, int 
                 }
             }
         }
-        epilogue_chunk<UP, NACC>(a, row0, c, f, s, sc0, sc1, x0, x1);
+        epilogue_chunk<UP, NACC>(a, row0, nreal, c, f, s, sc0, sc1, x0, x1);
     }
 }
 
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile uint32_t *abort_flag = misc + 1;
     int *prefix = reinterpret_cast<int *>(misc + 4);
     int *poff = prefix + 40;
+    int *roff = prefix + 80;   // unpadded offsets
     const int m_tiles = a.M / kBM;
 
     if (threadIdx.x == 0) {
@@ -211,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0u;
         prefix[0] = 0;
         for (int e = 0; e <= a.E; ++e) poff[e] = a.poff[e];
+        for (int e = 0; e <= a.E; ++e) roff[e] = a.offsets[e];
         for (int e = 0; e < a.E; ++e)
             prefix[e + 1] = prefix[e] + m_tiles * ((poff[e + 1] - poff[e]) / BN) * a.splits;
         fence_mbar_init();
@@ -399,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = m * kBM + q * 32 + lane;
             const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::ACC;
             const int row0 = poff[e] + n * BN;
+            const int nreal = roff[e + 1] - roff[e] - n * BN;   // real rows of this tile (may exceed BN)
             // per-channel scales here; the per-block format applied them while dequantising
             const float sc0 = a.kblock ? 1.f : __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
             const float sc1 = !UP ? 0.f : a.kblock ? 1.f : __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
@@ -443,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld16(tl + c, x0);
                     if constexpr (C::NACC == 2) tmem_ld16(tl + BN + c, x1);
                     tmem_wait_ld();
-                    epilogue_chunk<UP, C::NACC>(eo, row0, c, f, s, sc0, sc1, x0, x1);
+                    epilogue_chunk<UP, C::NACC>(eo, row0, nreal, c, f, s, sc0, sc1, x0, x1);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -452,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the tile's pieces are consecutive in the workspace
                 const float *p0 =
                     a.part + (static_cast<size_t>(wi.tile - wl.whole) * wl.P * kBM + q * 32 + lane) * C::ACC;
-                finish_pieces<UP, BN, C::NACC, C::ACC>(eo, p0, wl.P, c0, c1, row0, f, s, sc0, sc1);
+                finish_pieces<UP, BN, C::NACC, C::ACC>(eo, p0, wl.P, c0, c1, row0, nreal, f, s, sc0, sc1);
             }
             PS_ADD(c_ework, t1);
         }

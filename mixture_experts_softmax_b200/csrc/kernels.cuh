@@ -61,7 +61,9 @@ struct GemmArgs {
     int K;                      // reduction length (d for UP, F for DOWN)
     int ksteps;                 // k-steps of kBK per split
     int splits;                 // K-splits (DOWN); 1 for UP
-    const int *poff;            // [E+1]
+    const int *poff;            // [E+1] expert segments, padded to tile width
+    const int *offsets;         // [E+1] the same without padding: real rows of expert e are the first
+                                //       offsets[e+1] - offsets[e] rows of its segment
     const int *rperm;           // [rows]
     const float *gate;          // [T, 2]
     const __nv_bfloat16 *s0;    // [E, M]

@@ -408,6 +408,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.ksteps = h->d / kstage_of(h, true, bn);
     up.splits = 1;
     up.poff = poff;
+    up.offsets = rw + L.offsets;
     up.rperm = rperm;
     up.gate = gate;
     up.s0 = static_cast<const __nv_bfloat16 *>(s_lin);
