@@ -21,20 +21,35 @@ __device__ __forceinline__ void add4(float4 &a, const float4 &b)
     a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
 }
 
-// fixed-order sum of one token's slots for 4 consecutive features
+// fixed-order sum of one token's slots for 4 consecutive features.  The split loop runs to
+// the compile-time maximum MAXS with the unused splits predicated off, so that all the loads
+// of a chunk are in flight together instead of one L2 round trip per split.
+template <int MAXS>
 __device__ __forceinline__ float4 slot_sum(const CombineArgs &a, int t, int c)
 {
     const size_t plane = static_cast<size_t>(a.T) * 2 * a.d;
     const float *p = a.slots + (static_cast<size_t>(t) * 2) * a.d + c;
-    float4 y0 = ld4(p), y1 = ld4(p + a.d);
-    for (int s = 1; s < a.splits; ++s) {
-        add4(y0, ld4(p + s * plane));
-        add4(y1, ld4(p + s * plane + a.d));
+    float4 v0[MAXS], v1[MAXS];
+#pragma unroll
+    for (int s = 0; s < MAXS; ++s) {
+        if (s < a.splits) {
+            v0[s] = ld4(p + s * plane);
+            v1[s] = ld4(p + s * plane + a.d);
+        }
+    }
+    float4 y0 = v0[0], y1 = v1[0];
+#pragma unroll
+    for (int s = 1; s < MAXS; ++s) {
+        if (s < a.splits) {
+            add4(y0, v0[s]);
+            add4(y1, v1[s]);
+        }
     }
     add4(y0, y1);
     return y0;
 }
 
+template <int MAXS>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 {
     const int per_row = a.d >> 2;
@@ -43,7 +58,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
         const int t = static_cast<int>(i / per_row), c = static_cast<int>(i % per_row) * 4;
         // a padding token (expert -1) has no slots: its output row is 0
-        const float4 y = __ldg(a.idx + 2 * t) < 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : slot_sum(a, t, c);
+        const float4 y = __ldg(a.idx + 2 * t) < 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : slot_sum<MAXS>(a, t, c);
         __nv_bfloat162 lo = __floats2bfloat162_rn(y.x, y.y), hi = __floats2bfloat162_rn(y.z, y.w);
         uint2 v;
         v.x = *reinterpret_cast<uint32_t *>(&lo);
@@ -53,6 +68,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 }
 
 // one block per token: y = sum of slots; h <- bf16( h + y * rsqrt(mean(y^2) + eps) * g_post )
+template <int MAXS>
 __global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
 {
     __shared__ float red[8];
@@ -60,7 +76,7 @@ __global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
     if (__ldg(a.idx + 2 * t) < 0) return;   // a padding token: the residual row passes through unchanged
     float ss = 0.f;
     for (int c = threadIdx.x * 4; c < a.d; c += blockDim.x * 4) {
-        const float4 y = slot_sum(a, t, c);
+        const float4 y = slot_sum<MAXS>(a, t, c);
         ss = fmaf(y.x, y.x, fmaf(y.y, y.y, fmaf(y.z, y.z, fmaf(y.w, y.w, ss))));
     }
 #pragma unroll
@@ -73,7 +89,7 @@ __global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
     const float r = rsqrtf(tot / static_cast<float>(a.d) + a.eps);
     __nv_bfloat16 *hr = a.h_io + static_cast<size_t>(t) * a.d;
     for (int c = threadIdx.x * 4; c < a.d; c += blockDim.x * 4) {
-        const float4 y = slot_sum(a, t, c);
+        const float4 y = slot_sum<MAXS>(a, t, c);
         const float yv[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -88,13 +104,20 @@ __global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s)
 {
     if (a.T <= 0) return cudaSuccess;
+    // one split (large batches): the plain loop; several: all split loads in flight together
     if (a.h_io) {
-        combine_postnorm_kernel<<<a.T, 256, 0, s>>>(a);
+        if (a.splits == 1)
+            combine_postnorm_kernel<1><<<a.T, 256, 0, s>>>(a);
+        else
+            combine_postnorm_kernel<kMaxSplits><<<a.T, 256, 0, s>>>(a);
     } else {
         const size_t n = static_cast<size_t>(a.T) * (a.d >> 2);
         const size_t want = (n + 255) / 256;
         const int grid = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
-        combine_kernel<<<grid, 256, 0, s>>>(a);
+        if (a.splits == 1)
+            combine_kernel<1><<<grid, 256, 0, s>>>(a);
+        else
+            combine_kernel<kMaxSplits><<<grid, 256, 0, s>>>(a);
     }
     return cudaGetLastError();
 }
