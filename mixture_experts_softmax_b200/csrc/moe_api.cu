@@ -251,11 +251,13 @@ int encode_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *ptr
 
 // int8 weight descriptor.  [E, in, out] layout: rows = E*in, box = 64 k-rows x 128 features.
 // [E, out, in] (packed) layout: rows = E*out, box = 128 feature-rows x 128 k.
-int weight_map(moe_ctx *h, const void *ptr, int kind, const CUtensorMap **out)
+// The tensor map of a weight, from the handle's cache (encoded on first use).  The map is
+// copied out: a pointer into the cache would dangle once a later insertion moves it.
+int weight_map(moe_ctx *h, const void *ptr, int kind, CUtensorMap *out)
 {
     for (auto &w : h->wmaps)
         if (w.ptr == ptr && w.kind == kind && w.layout == h->layout) {
-            *out = &w.map;
+            *out = w.map;
             return MOE_OK;
         }
     WeightMap w;
@@ -273,7 +275,7 @@ int weight_map(moe_ctx *h, const void *ptr, int kind, const CUtensorMap **out)
     if (rc != MOE_OK) return rc;
     if (h->wmaps.size() >= 64) h->wmaps.erase(h->wmaps.begin());
     h->wmaps.push_back(w);
-    *out = &h->wmaps.back().map;
+    *out = w.map;
     return MOE_OK;
 }
 
@@ -364,7 +366,8 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
 
     const bool ts = h->layout == MOE_LAYOUT_PACKED;
     if (h->kblock && !ts) return MOE_EUNSUPPORTED;   // block scales: TMEM-operand kernels only
-    const CUtensorMap *m_wl, *m_wv, *m_w1, *m_xp, *m_h;
+    CUtensorMap m_wl, m_wv, m_w1;
+    const CUtensorMap *m_xp, *m_h;   // in the handle's fixed arrays
     if ((rc = weight_map(h, w_lin, 0, &m_wl)) != MOE_OK) return rc;
     if ((rc = weight_map(h, w_v, 0, &m_wv)) != MOE_OK) return rc;
     if ((rc = weight_map(h, w_1, 1, &m_w1)) != MOE_OK) return rc;
@@ -391,7 +394,11 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     GatherArgs ga{h->d, g_pre ? u : routed, static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
     if (small) {
         unsigned int *ticket = reinterpret_cast<unsigned int *>(h->err + kCtlRouteTicket);
-        if (timed(h, K_ROUTE_SMALL, s, [&] { return launch_route_small(ra, da, ga, ticket, s); }) != cudaSuccess)
+        // the partial logits go to the combine's slot buffer, which is free until the down-projection
+        float *part = static_cast<float *>(h->b_slots.ptr);
+        const int S = route_small_slices(T, h->d, h->num_sms);
+        if (timed(h, K_ROUTE_SMALL, s, [&] { return launch_route_small(ra, da, ga, part, S, ticket, s); }) !=
+            cudaSuccess)
             return MOE_ECUDA;
     } else {
         if (timed(h, K_ROUTER, s, [&] { return launch_router(ra, s); }) != cudaSuccess) return MOE_ECUDA;
@@ -422,8 +429,8 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
         up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
     }
     if (timed(h, K_UP, s, [&] {
-            return ts ? launch_gemm_up_ts(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s)
-                      : launch_gemm_up(bn, *m_wl, *m_wv, *m_xp, up, h->num_sms, s);
+            return ts ? launch_gemm_up_ts(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s)
+                      : launch_gemm_up(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s);
         }) != cudaSuccess)
         return MOE_ECUDA;
 
@@ -437,8 +444,8 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     dn.h = nullptr;
     dn.slots = static_cast<float *>(h->b_slots.ptr);
     if (timed(h, K_DOWN, s, [&] {
-            return ts ? launch_gemm_down_ts(bn, *m_w1, *m_h, dn, h->num_sms, s)
-                      : launch_gemm_down(bn, *m_w1, *m_h, dn, h->num_sms, s);
+            return ts ? launch_gemm_down_ts(bn, m_w1, *m_h, dn, h->num_sms, s)
+                      : launch_gemm_down(bn, m_w1, *m_h, dn, h->num_sms, s);
         }) != cudaSuccess)
         return MOE_ECUDA;
 
