@@ -145,36 +145,126 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs g, int T, const 
     gather_rows(g, T, slot_of_route, blockIdx.x, gridDim.x);
 }
 
-// Small batches in one launch: block t computes token t's logits and top-2 (route_token);
-// every block then takes a ticket, and the block holding the last one, which sees every
-// block's expert choice, runs the dispatch and gathers the 2T rows.  The ticket counter
-// is a workspace word that the last block sets back to 0 for the next launch.
+// The dispatch of T <= kFusedMaxT tokens by one block whose expert indices are already in
+// shared memory (s_idx[2t + j], -1 for a padding token's routes).  A route's rank within its
+// expert is the number of routes with a smaller id and the same expert: the two routes of a
+// token go to different experts, so this is the token-ordered stable grouping that
+// dispatch_block forms.  s_slot receives slot_of_route.
+__device__ __forceinline__ void dispatch_small(const DispatchArgs &a, const int *s_idx, int *s_slot)
+{
+    __shared__ int s_cnt[kMaxE], s_off[kMaxE + 1], s_poff[kMaxE + 1];
+    const int tid = threadIdx.x, R = 2 * a.T, E = a.E;
+    if (tid < E) {
+        int n = 0;
+        for (int r = 0; r < R; ++r) n += s_idx[r] == tid;
+        s_cnt[tid] = n;
+        a.counts[tid] = n;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        s_off[0] = 0;
+        s_poff[0] = 0;
+        for (int e = 0; e < E; ++e) {
+            s_off[e + 1] = s_off[e] + s_cnt[e];
+            s_poff[e + 1] = s_poff[e] + (s_cnt[e] + a.bn - 1) / a.bn * a.bn;
+        }
+    }
+    __syncthreads();
+    if (tid <= E) { a.offsets[tid] = s_off[tid]; a.poff[tid] = s_poff[tid]; }
+    if (tid < R) {
+        const int e = s_idx[tid];
+        int slot = -1;
+        if (e >= 0) {
+            int rank = 0;
+            for (int r = 0; r < tid; ++r) rank += s_idx[r] == e;
+            a.perm[s_off[e] + rank] = tid;
+            a.rperm[s_poff[e] + rank] = tid;
+            slot = s_poff[e] + rank;
+        }
+        a.slot_of_route[tid] = slot;
+        s_slot[tid] = slot;
+    }
+    for (int e = 0; e < E; ++e)   // padding rows of every expert segment carry route id -1
+        for (int r = s_poff[e] + s_cnt[e] + tid; r < s_poff[e + 1]; r += blockDim.x) a.rperm[r] = -1;
+    __syncthreads();
+}
+
+// Small batches in one launch.  Block b takes slice b % S of token b / S's row (S row
+// slices per token, S * T blocks) and writes the slice's partial logits to part[b][E]
+// (route_slice).  Every block then takes a ticket; the block holding the last one sums
+// each token's S partials in slice order, picks the top-2 and gates, dispatches from
+// shared memory and, when ga.xp is set, gathers the 2T rows.  The ticket counter is a
+// workspace word that the last block sets back to 0 for the next launch.
 __global__ void __launch_bounds__(kRouteTokenThreads) route_small_kernel(RouteArgs ra, DispatchArgs da, GatherArgs ga,
-                                                                          unsigned int *ticket)
+                                                                          float *part, int S, unsigned int *ticket)
 {
     __shared__ bool s_last;
-    route_token(ra, blockIdx.x);
-    __threadfence();   // this block's idx / gate before its ticket
+    __shared__ float s_logit[kFusedMaxT][kExperts];
+    __shared__ int s_idx[2 * kFusedMaxT], s_slot[2 * kFusedMaxT];
+    const int t = blockIdx.x / S, sl = blockIdx.x - t * S;
+    if (!is_padding(ra, t)) {   // uniform over the block
+        const int per = (ra.d >> 3) / S;
+        float acc[kExperts];
+        route_slice(ra, t, sl * per, sl == S - 1 ? (ra.d >> 3) : (sl + 1) * per, acc);
+        if (threadIdx.x == 0) {
+#pragma unroll
+            for (int e = 0; e < kExperts; ++e) part[blockIdx.x * kExperts + e] = acc[e];
+        }
+    }
+    __threadfence();   // this block's partials (and u) before its ticket
     __syncthreads();
     if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
     __syncthreads();
     if (!s_last) return;
-    __threadfence();   // every other block's idx / gate is visible after their tickets
+    __threadfence();   // every other block's partials are visible after their tickets
+    const int T = ra.T;
     if (threadIdx.x == 0) *ticket = 0u;
-    dispatch_block<kRouteTokenThreads>(da);
-    __syncthreads();   // slot_of_route of this block's dispatch, read back below
-    gather_rows(ga, da.T, da.slot_of_route, 0, 1);
+    if (threadIdx.x < T * kExperts) {   // fixed order: slices 0 .. S-1
+        const int tt = threadIdx.x / kExperts, e = threadIdx.x % kExperts;
+        float v = 0.f;
+        for (int q = 0; q < S; ++q) v += __ldcg(part + (tt * S + q) * kExperts + e);
+        s_logit[tt][e] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < T) {
+        const int tt = threadIdx.x;
+        if (is_padding(ra, tt)) {
+            s_idx[2 * tt] = -1;
+            s_idx[2 * tt + 1] = -1;
+            write_padding_route(tt, ra.idx, ra.gate);
+        } else {
+            float acc[kExperts], g[2];
+#pragma unroll
+            for (int e = 0; e < kExperts; ++e) acc[e] = s_logit[tt][e];
+            select_top2(acc, ra.bias, 0, s_idx + 2 * tt, g);
+            ra.idx[2 * tt] = s_idx[2 * tt];
+            ra.idx[2 * tt + 1] = s_idx[2 * tt + 1];
+            ra.gate[2 * tt] = g[0];
+            ra.gate[2 * tt + 1] = g[1];
+        }
+    }
+    __syncthreads();
+    dispatch_small(da, s_idx, s_slot);
+    if (ga.xp) gather_rows(ga, T, s_slot, 0, 1);
 }
 
 }  // namespace
 
 int route_small_max_tokens() { return kFusedMaxT; }
 
-cudaError_t launch_route_small(const RouteArgs &ra, const DispatchArgs &da, const GatherArgs &ga, unsigned int *ticket,
-                               cudaStream_t s)
+int route_small_slices(int T, int d, int num_sms)
 {
-    if (ra.T <= 0 || ra.T > kFusedMaxT) return cudaErrorInvalidValue;
-    route_small_kernel<<<ra.T, kRouteTokenThreads, 0, s>>>(ra, da, ga, ticket);
+    const int chunks = d >> 3;
+    int S = 1;   // row slices per token: the most that keep one wave and a warp's worth of chunks each
+    while (T * 2 * S <= num_sms && chunks % (2 * S) == 0 && chunks / (2 * S) >= 32) S *= 2;
+    return S;
+}
+
+cudaError_t launch_route_small(const RouteArgs &ra, const DispatchArgs &da, const GatherArgs &ga, float *part, int S,
+                               unsigned int *ticket, cudaStream_t s)
+{
+    if (ra.T <= 0 || ra.T > kFusedMaxT || S <= 0 || (ra.d >> 3) < S || da.E > kMaxE) return cudaErrorInvalidValue;
+    route_small_kernel<<<ra.T * S, kRouteTokenThreads, 0, s>>>(ra, da, ga, part, S, ticket);
     return cudaGetLastError();
 }
 

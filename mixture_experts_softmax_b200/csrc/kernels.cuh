@@ -104,11 +104,14 @@ cudaError_t launch_router(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 // Xp[slot_of_route[r]] = x[r / 2] for the 2T routes
 cudaError_t launch_gather(const GatherArgs &a, int T, const int *slot_of_route, cudaStream_t s);
-// router + dispatch + gather in one launch for T <= route_small_max_tokens(); `ticket` is a
-// zero-initialised device word owned by the caller (left at 0 after the launch)
+// router + dispatch (+ gather when ga.xp is set) in one launch of T * S blocks for
+// T <= route_small_max_tokens(), S = route_small_slices(T, d, SMs) row slices per token;
+// `part` is fp32 scratch of T * S * 8 words, `ticket` a zero-initialised device word owned by
+// the caller (left at 0 after the launch)
 int route_small_max_tokens();
-cudaError_t launch_route_small(const RouteArgs &ra, const DispatchArgs &da, const GatherArgs &ga, unsigned int *ticket,
-                               cudaStream_t s);
+int route_small_slices(int T, int d, int num_sms);
+cudaError_t launch_route_small(const RouteArgs &ra, const DispatchArgs &da, const GatherArgs &ga, float *part, int S,
+                               unsigned int *ticket, cudaStream_t s);
 cudaError_t launch_gemm_up(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
                            const GemmArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_gemm_down(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,

@@ -154,4 +154,83 @@ __device__ __forceinline__ void route_token(const RouteArgs &a, int t)
     }
 }
 
+// The logits of token t over the chunks [c0, c1) of its row (8 elements per chunk), one
+// chunk per thread and pass: every thread's loads are issued together, the dot products
+// take the chunk's rows in order, and the block reduces in a fixed order (lane tree, then
+// the warps in order) into thread 0's `acc`.  With a.g_pre set the routed row is the
+// RMS-normalised u of the residual block: the sum of squares is taken over the whole row
+// (the same fixed order in every block that calls this for token t, so all of them get the
+// same scale), and the slice's chunks of u are formed, rounded to bf16, stored to a.u and
+// used.  Without a.g_pre and with a.u set, the slice's chunks of x are copied to a.u.
+__device__ __forceinline__ void route_slice(const RouteArgs &a, int t, int c0, int c1, float (&acc)[kExperts])
+{
+    constexpr int kWarps = kRouteTokenThreads / 32;
+    __shared__ float part[kWarps][kExperts];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * a.d);
+    const float4 *w4 = reinterpret_cast<const float4 *>(a.w);
+    uint4 *ur = a.u ? reinterpret_cast<uint4 *>(a.u + static_cast<size_t>(t) * a.d) : nullptr;
+#pragma unroll
+    for (int e = 0; e < kExperts; ++e) acc[e] = 0.f;
+    float r = 0.f;
+    if (a.g_pre) {
+        const int chunks = a.d >> 3;
+        float ss = 0.f;
+        for (int c = threadIdx.x; c < chunks; c += kRouteTokenThreads) {
+            const uint4 v = __ldg(xr + c);
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float lo = __uint_as_float(wv[q] << 16), hi = __uint_as_float(wv[q] & 0xffff0000u);
+                ss = fmaf(lo, lo, ss);
+                ss = fmaf(hi, hi, ss);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) part[warp][0] = ss;
+        __syncthreads();
+        float tot = 0.f;
+        for (int w = 0; w < kWarps; ++w) tot += part[w][0];
+        __syncthreads();   // part is reused for the logits below
+        r = rsqrtf(tot / static_cast<float>(a.d) + a.eps);
+    }
+    for (int c = c0 + threadIdx.x; c < c1; c += kRouteTokenThreads) {
+        uint4 v = __ldg(xr + c);
+        if (a.g_pre) {
+            const uint4 g = __ldg(reinterpret_cast<const uint4 *>(a.g_pre) + c);
+            const uint32_t hv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w};
+            uint32_t uv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float lo = __uint_as_float(hv[q] << 16) * r * __uint_as_float(gv[q] << 16);
+                const float hi = __uint_as_float(hv[q] & 0xffff0000u) * r * __uint_as_float(gv[q] & 0xffff0000u);
+                const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+                uv[q] = *reinterpret_cast<const uint32_t *>(&p);
+            }
+            v = make_uint4(uv[0], uv[1], uv[2], uv[3]);
+        }
+        if (ur) ur[c] = v;
+        dot8(v, w4, c * 8, acc);
+    }
+#pragma unroll
+    for (int e = 0; e < kExperts; ++e) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int e = 0; e < kExperts; ++e) part[warp][e] = acc[e];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int e = 0; e < kExperts; ++e) {
+            float v = 0.f;
+            for (int w = 0; w < kWarps; ++w) v += part[w][e];
+            acc[e] = v;
+        }
+    }
+}
+
 }  // namespace moe
