@@ -270,6 +270,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             PS_FLUSH(SB + 1, c_wait);
         }
         __syncwarp();
+    } else if (UP && BN <= 32 && warp == kWarpTmaB && a.gather) {
+        // ---- small batches: the activation rows straight from the routed rows -----------
+        // tmB covers the routed rows [T, d] with one-row boxes.  Lane q copies tile rows
+        // 4q .. 4q+3 (tokens rperm >> 1) with one four-row gather per 64-wide box, into the
+        // place the tiled load gives those rows; rows from nreal on repeat row 0's token.
+        // Each accumulator column depends on its own B row only, and the epilogue skips the
+        // columns from nreal on.
+        const uint64_t pol = l2_policy_evict_last();
+        uint32_t st = 0, ph = 0, issued = 0, par = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < wl.items; item += gridDim.x) {
+            if (__shfl_sync(0xffffffffu, lane == 0 ? static_cast<int>(*abort_flag) : 0, 0)) break;
+            const WorkItem wi = work_item(wl, item, a.ksteps);
+            int e, m, n, s;
+            decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+            const int kb = s * a.ksteps;
+            const int row = poff[e] + n * BN;
+            const int nreal = min(BN, roff[e + 1] - roff[e] - n * BN);
+            const int ngroups = (nreal + 3) >> 2;
+            const int tok = lane < nreal ? (__ldg(a.rperm + row + lane) >> 1) : -1;
+            const int tok0 = __shfl_sync(0xffffffffu, tok, 0);
+            int g[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int v = __shfl_sync(0xffffffffu, tok, (4 * lane + i) & 31);
+                g[i] = 4 * lane + i < nreal ? v : tok0;
+            }
+            for (int ks = wi.k0; ks < wi.k1; ++ks) {
+                if (lane == 0) ok = w.wait(op_empty(st), ph ^ 1u, 2);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (lane == 0) mbar_arrive_expect_tx(b_full(st), static_cast<uint32_t>(ngroups) * 4 * C::KSTAGE * 2);
+                __syncwarp();
+                const uint32_t dst = sbase + C::OFF_B + st * C::BBYTES + lane * 4 * 128;
+                const int x = (kb + ks) * C::KSTAGE;
+                if (lane < ngroups) {
+#pragma unroll
+                    for (int j = 0; j < C::KSTAGE / 64; ++j)
+                        tma_gather4(dst + j * BN * 128, &tmB, b_full(st), x + 64 * j, g[0], g[1], g[2], g[3], pol);
+                }
+                issued |= 1u << st;
+                par = (par & ~(1u << st)) | (ph << st);
+                if (++st == C::S2) { st = 0; ph ^= 1u; }
+            }
+        }
+        if (lane == 0)
+            for (int s = 0; s < C::S2; ++s)
+                if (issued & (1u << s)) wait_drain(b_full(s), (par >> s) & 1u);
+        __syncwarp();
     } else if (warp == kWarpTmaB) {
         // ---- bf16 activation tiles [BN r x 128 k] (two 64-wide boxes) -> operand ring --
         if (lane == 0) {

@@ -79,6 +79,10 @@ struct GemmArgs {
     // last-wave pieces (TMEM-operand kernels): partial accumulators and per-tile tickets
     float *part;                // [gridDim.x, 128, accumulator columns] fp32, or nullptr: no pieces
     unsigned int *tickets;      // [gridDim.x], zero, left zero by every launch that completes
+    // TMEM-operand up-projection with tiles of at most 32 rows: 1 = the B map covers the routed
+    // rows [T, K] with one-row boxes and each tile row is loaded from row rperm >> 1 of it
+    // (no gathered copy); 0 = the B map covers the gathered rows [rows, K]
+    int gather;
 };
 
 struct CombineArgs {

@@ -61,6 +61,9 @@ struct moe_ctx {
     // TMA descriptors
     std::vector<WeightMap> wmaps;
     CUtensorMap xp_map[4], h_map[4];
+    CUtensorMap stage_map;              // b_stage as bf16 [rows, d], one-row boxes (small-batch B rows)
+    const void *stage_map_ptr = nullptr;
+    size_t stage_map_bytes = 0;
     int xp_map_gen[4] = {-1, -1, -1, -1}, h_map_gen[4] = {-1, -1, -1, -1};
 
     const float *bias = nullptr;
@@ -300,6 +303,21 @@ int act_maps(moe_ctx *h, int bn, const CUtensorMap **xp, const CUtensorMap **hm)
     return MOE_OK;
 }
 
+// the routed rows of a small batch (b_stage as bf16 [rows, d]) with one-row boxes of kBK
+// columns, for the up-projection's per-row loads
+int stage_map(moe_ctx *h, const CUtensorMap **out)
+{
+    if (h->stage_map_ptr != h->b_stage.ptr || h->stage_map_bytes != h->b_stage.bytes) {
+        const uint64_t rows = h->b_stage.bytes / (static_cast<uint64_t>(h->d) * 2);
+        const int rc = encode_2d(&h->stage_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->b_stage.ptr, h->d, rows, kBK, 1);
+        if (rc != MOE_OK) return rc;
+        h->stage_map_ptr = h->b_stage.ptr;
+        h->stage_map_bytes = h->b_stage.bytes;
+    }
+    *out = &h->stage_map;
+    return MOE_OK;
+}
+
 cudaEvent_t take_event(moe_ctx *h)
 {
     if (!h->event_pool.empty()) {
@@ -392,6 +410,16 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     }
     DispatchArgs da{T, h->E, bn, idx, rw + L.counts, rw + L.offsets, poff, rw + L.perm, rperm, rw + L.slot};
     GatherArgs ga{h->d, g_pre ? u : routed, static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
+    // small batches on the TMEM-operand kernels: the routing launch leaves the routed rows in
+    // the staging buffer (copied there unless they already are) and the up-projection loads
+    // its B rows from it, so nothing is gathered
+    const bool gather_in_gemm = small && ts;
+    const CUtensorMap *m_b = m_xp;
+    if (gather_in_gemm) {
+        if ((rc = stage_map(h, &m_b)) != MOE_OK) return rc;
+        if (!g_pre && routed != u) ra.u = u;
+        ga.xp = nullptr;
+    }
     if (small) {
         unsigned int *ticket = reinterpret_cast<unsigned int *>(h->err + kCtlRouteTicket);
         // the partial logits go to the combine's slot buffer, which is free until the down-projection
@@ -424,17 +452,19 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.err = h->err;
     up.timeout_ns = h->timeout_ns;
     up.kblock = h->kblock;
+    up.gather = gather_in_gemm ? 1 : 0;
     if (ts) {
         up.part = static_cast<float *>(h->b_part.ptr);
         up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
     }
     if (timed(h, K_UP, s, [&] {
-            return ts ? launch_gemm_up_ts(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s)
+            return ts ? launch_gemm_up_ts(bn, m_wl, m_wv, *m_b, up, h->num_sms, s)
                       : launch_gemm_up(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s);
         }) != cudaSuccess)
         return MOE_ECUDA;
 
     GemmArgs dn = up;
+    dn.gather = 0;
     dn.M = h->d;
     dn.K = h->F;
     dn.splits = splits;
