@@ -187,23 +187,30 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_source_hash():
+GEMM_SOURCES = {"packed": ("gemm_ts.cu", "gemm_common.cuh", "ptx.cuh", "kernels.cuh"),
+                "in_out": ("gemm.cu", "gemm_common.cuh", "ptx.cuh", "kernels.cuh")}
+
+
+def kernel_source_hash(layout):
+    """Hash of the GEMM sources of a weight layout: a recorded DRAM-traffic figure holds only for them."""
     h = hashlib.sha256()
-    for name in ("gemm.cu", "ptx.cuh", "kernels.cuh"):
+    for name in GEMM_SOURCES[layout]:
         with open(os.path.join(ROOT, "mixture_experts_softmax_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, kernel):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel has not changed since."""
+def recorded_traffic(workload, layout, kernel, variant):
+    """DRAM bytes per full-size launch from the committed ncu summary (profiles/traffic.json),
+    or None: no record for this workload, a variant of it (resized, other scale format), or
+    GEMM sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+    if variant or not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    ent = rec.get(f"{workload}/{kernel}")
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    ent = rec.get(f"{workload}/{layout}/{kernel}")
+    if not ent or ent.get("source_hash") != kernel_source_hash(layout):
         return None
     return ent.get("bytes_per_launch")
 
@@ -233,6 +240,7 @@ def run_native(args, world, rank, local):
     if args.tokens or args.ffn:
         import dataclasses
         w = dataclasses.replace(w, T=args.tokens or w.T, F=args.ffn or w.F, name=w.name + "_resized")
+    variant = bool(args.tokens or args.ffn or args.scale_block)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     K, W = args.steps, args.warmup
@@ -361,17 +369,15 @@ def run_native(args, world, rank, local):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "frac_of_burst": achieved / peaks["bf16_tflops"],
                 "kernel": "up_proj", "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
-                "traffic": recorded_traffic(args.workload, "up_proj"),
+                "traffic": recorded_traffic(args.workload, args.layout, "up_proj", variant),
                 "algorithmic_flops_per_launch": work["up_flops"], "launch_ms": up_ms}
     else:
-        nb = work["up_bytes"] * (w.blocks or 1)
         achieved = work["up_bytes"] / (up_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "kernel": "up_proj", "peak_source": f"{peak_src} hbm_gbs (copy)",
-                "traffic": recorded_traffic(args.workload, "up_proj"),
+                "traffic": recorded_traffic(args.workload, args.layout, "up_proj", variant),
                 "algorithmic_bytes_per_launch": work["up_bytes"], "launch_ms": up_ms}
-        del nb
     layer_bytes = (work["up_bytes"] + work["dn_bytes"]) * (w.blocks or 1)
     layer_roof = {"bytes_per_step": layer_bytes, "GBps": layer_bytes / (ms / 1e3) / 1e9,
                   "frac_hbm": layer_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
