@@ -98,16 +98,19 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t par)
         if (global_timer_ns() - t0 > 1000000000ull) return;
 }
 
+// tile index -> expert e, output tile m, route tile n, reduction split s: splits vary
+// fastest, then route tiles, then output tiles, expert after expert.  A route tile covers
+// `pair` consecutive BN-row segments of its expert (the expert's last tile may cover fewer).
 template <int BN>
 __device__ __forceinline__ void decode_tile(int tile, const int *prefix, const int *poff, int m_tiles,
-                                            int splits, int &e, int &m, int &n, int &s)
+                                            int splits, int &e, int &m, int &n, int &s, int pair = 1)
 {
     e = 0;
     while (tile >= prefix[e + 1]) ++e;
     int local = tile - prefix[e];
     s = local % splits;
     local /= splits;
-    const int nt = (poff[e + 1] - poff[e]) / BN;
+    const int nt = ((poff[e + 1] - poff[e]) / BN + pair - 1) / pair;   // tiles of `pair` BN-row segments
     n = local % nt;
     m = local / nt;
 }

@@ -48,25 +48,32 @@ static_assert(kWarpConv0 + kConvWarps == kThreads / 32 && kWarpEpi0 + kEpiWarps 
 template <bool UP, int BN>
 struct CfgTS {
     static constexpr bool K2 = !UP && BN <= 64;             // two k-boxes per stage
+    // The 128-route down-projection takes route tiles of two consecutive 128-row segments of an
+    // expert: one N = 256 MMA per K slice (N = 128 for an expert's odd last segment), so each
+    // converted weight box serves 256 routes and a stage carries 1024 MMA cycles against
+    // 160 KB of shared-memory traffic, the balance of the up-projection.
+    static constexpr bool WIDE = !UP && BN == 128;
+    static constexpr int PAIR = WIDE ? 2 : 1;               // BN-row segments per route tile
+    static constexpr int TN = PAIR * BN;                    // MMA N (accumulator columns) of a full tile
     static constexpr int NB = UP ? 2 : (K2 ? 2 : 1);        // weight boxes per stage
     static constexpr int KSTAGE = K2 ? 2 * kBKT : kBKT;     // reduction elements per stage
     static constexpr int KP = kConvWarps / 4 / NB;          // converter warps per (quadrant, box)
     static constexpr int CH = (kBKT / 16) / KP;             // 16-byte chunks per converter thread and stage
     static constexpr int STG = NB * kBM * kBKT;             // int8 staging bytes per stage
-    static constexpr int BBYTES = BN * KSTAGE * 2;          // bf16 activation bytes per stage
+    static constexpr int BBYTES = TN * KSTAGE * 2;          // bf16 activation bytes per stage
     // Two MMA issuers, each into an accumulator of its own: per box of a stage for the
     // up-projection (one accumulator per matrix anyway) and the narrow down-projection (one per
     // k-box); per half of the stage's 8 K slices for the 128-route down-projection, whose stage
     // holds one box (KSPLIT).  The epilogue sums a down-projection's two accumulators.  The
     // converter warps keep every SM sub-partition's issue slots busy, and a single issuing
     // thread, which spends several instructions per MMA, then falls behind the tensor core.
-    static constexpr bool KSPLIT = !UP && !K2;
+    static constexpr bool KSPLIT = !UP && !K2 && !WIDE;
     static constexpr bool DUAL = UP || (K2 && BN <= 32) || KSPLIT;
     static constexpr int NACC = DUAL ? 2 : 1;               // accumulators per tile
-    static constexpr int ACC = NACC * BN;                   // TMEM columns of one accumulator buffer
-    static constexpr int NDB = (NACC * BN > 128) ? 1 : 2;   // accumulator buffers in TMEM
+    static constexpr int ACC = NACC * TN;                   // TMEM columns of one accumulator buffer
+    static constexpr int NDB = ACC > 128 ? 1 : 2;           // accumulator buffers in TMEM
     static constexpr int A_COLS = NB * kBKT / 2;            // TMEM columns of one A stage
-    static constexpr int S2 = cmin(4, (512 - NDB * ACC) / A_COLS);   // A (TMEM) + B (smem) ring
+    static constexpr int S2 = cmin(cmin(4, (512 - NDB * ACC) / A_COLS), (kSmemBudget - 2 * STG) / BBYTES);   // A (TMEM) + B (smem) ring
     static constexpr int S1 = cmin(12, (kSmemBudget - S2 * BBYTES) / STG);   // int8 staging ring
     static constexpr int A_BASE = NDB * ACC;                // first TMEM column of the A ring
     static constexpr int TMEM_COLS = pow2_at_least(NDB * ACC + S2 * A_COLS);
@@ -82,7 +89,7 @@ struct CfgTS {
     static_assert(SMEM <= 227 * 1024, "shared memory over the per-CTA limit");
     static_assert(TMEM_COLS <= 512, "TMEM has 512 columns");
     static_assert(KP >= 1 && CH * KP == kBKT / 16, "converter warps must split the 8 chunks of a row");
-    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is 16..256 in steps of 16");
+    static_assert(TN % 16 == 0 && BN >= 16 && TN <= 256, "UMMA N for M=128 is 16..256 in steps of 16");
 };
 
 // kind::f16 instruction descriptor: D fp32, A and B bf16, both K-major, M = 128.
@@ -215,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e <= a.E; ++e) poff[e] = a.poff[e];
         for (int e = 0; e <= a.E; ++e) roff[e] = a.offsets[e];
         for (int e = 0; e < a.E; ++e)
-            prefix[e + 1] = prefix[e] + m_tiles * ((poff[e + 1] - poff[e]) / BN) * a.splits;
+            prefix[e + 1] = prefix[e] + m_tiles * (((poff[e + 1] - poff[e]) / BN + C::PAIR - 1) / C::PAIR) * a.splits;
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -246,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int item = blockIdx.x; item < wl.items && !*abort_flag; item += gridDim.x) {
                 const WorkItem wi = work_item(wl, item, a.ksteps);
                 int e, m, n, s;
-                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s, C::PAIR);
                 const int kb = s * a.ksteps;
                 const int y = e * a.M + m * kBM;
                 for (int ks = wi.k0; ks < wi.k1; ++ks) {
@@ -284,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (__shfl_sync(0xffffffffu, lane == 0 ? static_cast<int>(*abort_flag) : 0, 0)) break;
             const WorkItem wi = work_item(wl, item, a.ksteps);
             int e, m, n, s;
-            decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+            decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s, C::PAIR);
             const int kb = s * a.ksteps;
             const int row = poff[e] + n * BN;
             const int nreal = min(BN, roff[e + 1] - roff[e] - n * BN);
@@ -328,19 +335,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int item = blockIdx.x; item < wl.items && !*abort_flag; item += gridDim.x) {
                 const WorkItem wi = work_item(wl, item, a.ksteps);
                 int e, m, n, s;
-                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s, C::PAIR);
                 const int kb = s * a.ksteps;
-                const int row = poff[e] + n * BN;
+                const int row = poff[e] + n * C::TN;
+                const int nseg = min(C::PAIR, (poff[e + 1] - row) / BN);   // BN-row segments of the tile
                 for (int ks = wi.k0; ks < wi.k1; ++ks) {
                     PS_NOW(t0);
                     if (!w.wait(op_empty(st), ph ^ 1u, 2)) goto b_done;
                     PS_ADD(c_bwait, t0);
-                    mbar_arrive_expect_tx(b_full(st), C::BBYTES);
+                    mbar_arrive_expect_tx(b_full(st), static_cast<uint32_t>(nseg) * BN * C::KSTAGE * 2);
                     const uint32_t dst = sbase + C::OFF_B + st * C::BBYTES;
                     const int x = (kb + ks) * C::KSTAGE;
 #pragma unroll
-                    for (int j = 0; j < C::KSTAGE / 64; ++j)   // 64-element (128-byte) wide boxes
-                        tma_load_2d(dst + j * BN * 128, &tmB, b_full(st), x + 64 * j, row, pol);
+                    for (int j = 0; j < C::KSTAGE / 64; ++j)   // 64-element (128-byte) wide boxes of TN rows
+                        for (int g = 0; g < nseg; ++g)
+                            tma_load_2d(dst + (j * C::TN + g * BN) * 128, &tmB, b_full(st), x + 64 * j, row + g * BN,
+                                        pol);
                     issued |= 1u << st;
                     par = (par & ~(1u << st)) | (ph << st);
                     if (++st == C::S2) { st = 0; ph ^= 1u; }
@@ -357,7 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // with two issuers, issuer i takes box i of every stage into accumulator i
         const int mine = warp == kWarpMma ? 0 : 1;
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_ts<BN>();
             uint32_t st = 0, ph = 0;
             int it = 0;
             PS_VAR(c_acc);
@@ -366,6 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             PS_VAR(c_issue);
             for (int item = blockIdx.x; item < wl.items; item += gridDim.x, ++it) {
                 const WorkItem wi = work_item(wl, item, a.ksteps);
+                uint32_t idesc = idesc_ts<C::TN>();
+                if constexpr (C::WIDE) {   // an expert's odd last segment: N = BN
+                    int e, m, n, s;
+                    decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s, C::PAIR);
+                    if (poff[e + 1] - (poff[e] + n * C::TN) < C::TN) idesc = idesc_ts<BN>();
+                }
                 const int b = it % C::NDB;
                 const uint32_t aph = (it / C::NDB) & 1;
                 PS_NOW(t0);
@@ -397,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // consecutive ones
                             const int kg = (UP ? 0 : bx * (kBKT / 16)) + kk;
                             const uint64_t bdesc =
-                                desc_sw128(bbase + (kg >> 2) * (BN * 128) + (kg & 3) * 32, 16, 1024);
+                                desc_sw128(bbase + (kg >> 2) * (C::TN * 128) + (kg & 3) * 32, 16, 1024);
                             // the item's first MMA into an accumulator starts it
                             const int kr = ks - wi.k0;
                             const int kf = C::KSPLIT ? (kk & 3) : kk;
@@ -427,9 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tiles: the first four warps take all 16 columns, the others only hand the buffer back)
         const int q = warp & 3;
         const int hc = (warp - kWarpEpi0) >> 2;
-        constexpr int kCols = BN >= 32 ? BN / 2 : BN;
+        constexpr int kCols = BN >= 32 ? C::TN / 2 : BN;
         const int c0 = BN >= 32 ? hc * kCols : 0;
-        const int c1 = BN >= 32 || hc == 0 ? c0 + kCols : c0;
+        const int c1_full = BN >= 32 || hc == 0 ? c0 + kCols : c0;
         volatile uint32_t *last_flag = misc + 2;
         const EpiOut eo{a.rperm, a.gate, a.h, a.slots, a.M, a.T};
         auto epilogue_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
@@ -439,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int item = blockIdx.x; item < wl.items; item += gridDim.x, ++it) {
             const WorkItem wi = work_item(wl, item, a.ksteps);
             int e, m, n, s;
-            decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+            decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s, C::PAIR);
             const int b = it % C::NDB;
             const uint32_t aph = (it / C::NDB) & 1;
             PS_NOW(t0);
@@ -450,8 +465,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int f = m * kBM + q * 32 + lane;
             const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::ACC;
-            const int row0 = poff[e] + n * BN;
-            const int nreal = roff[e + 1] - roff[e] - n * BN;   // real rows of this tile (may exceed BN)
+            const int row0 = poff[e] + n * C::TN;
+            const int nreal = roff[e + 1] - roff[e] - n * C::TN;   // real rows of this tile (may exceed TN)
+            // a wide tile over an expert's odd last segment has BN columns
+            const int c1 = C::WIDE ? max(c0, min(c1_full, poff[e + 1] - row0)) : c1_full;
             // per-channel scales here; the per-block format applied them while dequantising
             const float sc0 = a.kblock ? 1.f : __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
             const float sc1 = !UP ? 0.f : a.kblock ? 1.f : __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
@@ -540,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const __nv_bfloat16 *srow = nullptr;
             if (a.kblock) {
                 int e, m, n, s;
-                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s);
+                decode_tile<BN>(wi.tile, prefix, poff, m_tiles, a.splits, e, m, n, s, C::PAIR);
                 const int k0 = s * a.ksteps * C::KSTAGE + (UP ? 0 : box * kBKT);
                 srow = ((UP && box == 1) ? a.s1 : a.s0) +
                        (static_cast<size_t>(e) * (a.K / kScaleBlock) + k0 / kScaleBlock) * a.M + m * kBM + fr;
