@@ -44,7 +44,7 @@ static_assert(kWarpConv0 + kConvWarps == kThreads / 32 && kWarpEpi0 + kEpiWarps 
 // Weight tiles are [128 features x 128 reduction elements] int8 "boxes" of 16 KB.  A pipeline
 // stage carries NB boxes: the up-projection one box of each of its two matrices (same k), the
 // down-projection with narrow tiles two consecutive k-boxes of its one matrix (so every stage
-// moves 32 KB), the down-projection with 128-route tiles one box.
+// moves 32 KB), the down-projection with 128-route (wide, 256-route) tiles one box.
 template <bool UP, int BN>
 struct CfgTS {
     static constexpr bool K2 = !UP && BN <= 64;             // two k-boxes per stage
@@ -61,14 +61,12 @@ struct CfgTS {
     static constexpr int CH = (kBKT / 16) / KP;             // 16-byte chunks per converter thread and stage
     static constexpr int STG = NB * kBM * kBKT;             // int8 staging bytes per stage
     static constexpr int BBYTES = TN * KSTAGE * 2;          // bf16 activation bytes per stage
-    // Two MMA issuers, each into an accumulator of its own: per box of a stage for the
-    // up-projection (one accumulator per matrix anyway) and the narrow down-projection (one per
-    // k-box); per half of the stage's 8 K slices for the 128-route down-projection, whose stage
-    // holds one box (KSPLIT).  The epilogue sums a down-projection's two accumulators.  The
-    // converter warps keep every SM sub-partition's issue slots busy, and a single issuing
-    // thread, which spends several instructions per MMA, then falls behind the tensor core.
-    static constexpr bool KSPLIT = !UP && !K2 && !WIDE;
-    static constexpr bool DUAL = UP || (K2 && BN <= 32) || KSPLIT;
+    // Two MMA issuers, one per box of a stage, each into an accumulator of its own: the
+    // up-projection (one accumulator per matrix anyway) and the narrowest down-projections (one
+    // per k-box; the epilogue sums the two).  The converter warps keep every SM sub-partition's
+    // issue slots busy, and a single issuing thread, which spends several instructions per MMA,
+    // then falls behind the tensor core.
+    static constexpr bool DUAL = UP || (K2 && BN <= 32);
     static constexpr int NACC = DUAL ? 2 : 1;               // accumulators per tile
     static constexpr int ACC = NACC * TN;                   // TMEM columns of one accumulator buffer
     static constexpr int NDB = ACC > 128 ? 1 : 2;           // accumulator buffers in TMEM
@@ -404,9 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int bx = 0; bx < C::NB; ++bx) {
 #pragma unroll
                         for (int kk = 0; kk < kBKT / 16; ++kk) {
-                            // issuer / accumulator of this MMA: the box, or the half of the K slices
-                            const int who = C::KSPLIT ? (kk >> 2) : bx;
-                            if (C::DUAL && who != mine) continue;
+                            // issuer / accumulator of this MMA: the box
+                            if (C::DUAL && bx != mine) continue;
                             // K slice of the stage's activation tile; both matrices of the
                             // up-projection use the same slices, the k-boxes of the down-projection
                             // consecutive ones
@@ -415,9 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 desc_sw128(bbase + (kg >> 2) * (C::TN * 128) + (kg & 3) * 32, 16, 1024);
                             // the item's first MMA into an accumulator starts it
                             const int kr = ks - wi.k0;
-                            const int kf = C::KSPLIT ? (kk & 3) : kk;
-                            const uint32_t acc = C::DUAL ? ((kr | kf) != 0) : ((kr | bx | kk) != 0);
-                            umma_bf16_ts(dcol + (C::DUAL ? who : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc,
+                            const uint32_t acc = C::DUAL ? ((kr | kk) != 0) : ((kr | bx | kk) != 0);
+                            umma_bf16_ts(dcol + (C::DUAL ? bx : 0) * BN, acol + bx * (kBKT / 2) + kk * 8, bdesc,
                                          idesc, acc);
                         }
                     }

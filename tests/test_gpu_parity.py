@@ -75,6 +75,17 @@ def test_tiny_all_routes_to_one_expert(m, tiny_inputs, tiny_handle):
     parity.check_output(run, layer, x, range(300), near, bias_cpu=bias)
 
 
+@pytest.mark.parametrize("T", [13, 16, 32])
+def test_tiny_small_batch_one_expert_full_tile(m, tiny_inputs, tiny_handle, T):
+    """Small batches with +100 on expert 3: that expert's tile holds all T routes (a full
+    16- or 32-row tile at T = 16, 32; a ragged one at 13), the other experts share the
+    second picks; covers the up-projection's own row gather at every fill level."""
+    bias = torch.tensor([0, 0, 0, 100.0, 0, 0, 0, 0])
+    run, layer, x, near = _run_tiny(m, tiny_handle, tiny_inputs, T, bias=bias)
+    assert (run.idx_h[:, 0] == 3).all()
+    parity.check_output(run, layer, x, range(T), near, bias_cpu=bias)
+
+
 def test_tiny_only_two_experts_used(m, tiny_inputs, tiny_handle):
     bias = torch.tensor([0, 0, 0, 0, 0, 60.0, 0, 50.0])
     run, layer, x, near = _run_tiny(m, tiny_handle, tiny_inputs, 200, bias=bias)
