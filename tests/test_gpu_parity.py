@@ -355,6 +355,28 @@ def test_large_T_sampled(m, grok_handle, grok_layer, name, T):
     parity.check_output(run, layer_cpu, x_cpu, toks, near, bias_cpu=bias)
 
 
+def test_wide_tiles_odd_segments_and_pieces(m, grok_handle, grok_layer):
+    """+100 on experts 0 and 1: both take all T = 1664 routes, 13 segments of 128 each, so the
+    down-projection's 256-route tiles end on an odd 128-route tile; the plan (2 K-splits,
+    2 experts * 48 * 7 * 2 = 1344 tiles on 148 CTAs) cuts the last wave of 12 tiles into 12
+    pieces each."""
+    h, layer, _ = grok_handle
+    _, layer_cpu = grok_layer
+    T = 1664
+    rc, bn, splits = m.moe_plan(h, T)
+    assert (rc, bn, splits) == (0, 128, 2)
+    g = moe_synth.generator(23, "cuda")
+    x = moe_synth.draw_tokens(T, 6144, g, "cuda")
+    bias = torch.tensor([100.0, 100.0, 0, 0, 0, 0, 0, 0])
+    run = parity.Run(h, x, layer, bias.cuda())
+    assert run.offsets_h.tolist() == [0, T, 2 * T] + [2 * T] * 6
+    x_cpu = x.cpu()
+    ref = oracle.route(x_cpu, layer_cpu["router_w"], bias)
+    near = parity.check_routing(run, ref, 8)
+    toks = parity.sample_tokens(run, T, 48)
+    parity.check_output(run, layer_cpu, x_cpu, toks, near, bias_cpu=bias)
+
+
 def test_stacked_blocks_per_block(m, grok_handle):
     """Four residual blocks, T=32: each block on the GPU is fed the oracle's residual
     stream (bf16) so that every block is compared on identical inputs."""
