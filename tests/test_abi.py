@@ -68,6 +68,7 @@ def test_plan(m):
         assert m.moe_plan(h, 8192)[:2] == (0, 128)
         assert m.moe_plan(h, 8)[2] == 8          # decode: the down-projection splits K
         assert m.moe_plan(h, 8192)[2] == 1       # prefill: enough tiles without splitting
+        assert m.moe_plan(h, 1664) == (0, 128, 2)   # the plan test_wide_tiles_odd_segments_and_pieces needs
         assert m.moe_plan(h, -1)[0] == m.MOE_EINVAL
     finally:
         m.moe_destroy(h)
