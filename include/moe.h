@@ -135,8 +135,8 @@ MOE_API int moe_set_scale_block(moe_handle h, int kb);
  *   x    bf16 [T, d]   input tokens
  *   out  bf16 [T, d]   output; must not overlap x or the weights
  * Weights and scales as in the layout block above.  T == 0 is a no-op.
- * Enqueues the router, dispatch, gather, up-projection, down-projection and
- * combine kernels on `stream` and returns.  Deterministic: the same inputs give
+ * Enqueues the routing (router, dispatch, gather; one launch for T <= 32),
+ * up-projection, down-projection and combine kernels on `stream` and returns.  Deterministic: the same inputs give
  * bit-identical outputs.  Device-side wait timeouts are reported later by
  * moe_sync_status.  Returns MOE_EINVAL on a bad argument, MOE_ENOMEM if the
  * workspace could not grow, MOE_ECUDA if a launch failed.
@@ -204,8 +204,10 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns);
  * moe_set_profiling(h, 1) starts recording around each kernel of every forward;
  * moe_get_kernel_times synchronises on those events and returns, per kernel id
  * (0 router, 1 dispatch, 2 gather, 3 up-projection, 4 down-projection,
- * 5 combine, 6 pre-norm, 7 small-batch routing: router, dispatch and gather in
- * one launch, used instead of 0-2 when T <= 32), the total milliseconds and the
+ * 5 combine, 6 pre-norm, 7 small-batch routing: router and dispatch in one
+ * launch, used instead of 0-2 when T <= 32; in MOE_LAYOUT_PACKED the
+ * up-projection then loads the routed rows itself, in MOE_LAYOUT_IN_OUT that
+ * launch also gathers them), the total milliseconds and the
  * launch count since the previous call, then resets them.  n = capacity of
  * ms/launches (8 suffices).
  */
