@@ -15,12 +15,15 @@ Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``
 * ``expert_ffn``   pinned: numpy float64 dense gated FFN (library matmul).
 * ``forward``      pinned: forced-expert and closed-form-gate reductions, permutation
                    invariance, zero input, linearity in the output scale.
-* ``rmsnorm``      pinned: unit-RMS property, scale invariance.
+* ``rmsnorm``      pinned: unit-RMS property, scale invariance, the closed form of a
+                   constant row (which fixes where eps enters).
+* ``block_chain``  pinned: power-of-two scalings that the pre-norm, the post-norm, the
+                   gains and the residual add each fix exactly.
 * ``round_bf16``   pinned: torch's fp32 -> bf16 round-to-nearest-even.
-* ``gelu``         tanh form pinned by its odd-part identity and its distance to the
-                   exact (erf) GELU; the choice of the tanh form over the erf form
-                   is a reading, and the two differ by < 1e-3 -- at that level the
-                   GELU variant is parity unpinned.
+* ``gelu``         tanh form pinned against torch's tanh-approximate GELU (and by its
+                   odd-part identity); the erf form against math.erf.  Choosing the
+                   tanh form is a reading of the pages (they say "gelu" only); the two
+                   forms differ by < 1e-3.
 """
 from __future__ import annotations
 
@@ -178,6 +181,38 @@ def dispatch(idx, E: int):
     return counts, offsets, perm
 
 
+def check_layer(layer, d: Optional[int] = None) -> tuple:
+    """Shapes of one layer in the [E, in, out] orientation -> (E, d, F, kb); raises ValueError
+    when the tensors do not fit together (for example a layer whose weights were transposed
+    to another layout, or scales of another matrix)."""
+    shp = {k: tuple(layer[k].shape) for k in ("router_w", "wl", "sl", "wv", "sv", "w1", "s1")}
+    if len(shp["wl"]) != 3:
+        raise ValueError(f"wl must be [E, d, F], got {shp['wl']}")
+    E, dd, F = shp["wl"]
+    if d is not None and dd != d:
+        raise ValueError(f"wl is [E, {dd}, F] but the tokens have width {d} (weights in another layout?)")
+    if shp["wv"] != (E, dd, F):
+        raise ValueError(f"wv must be {(E, dd, F)}, got {shp['wv']}")
+    if shp["w1"] != (E, F, dd):
+        raise ValueError(f"w1 must be {(E, F, dd)}, got {shp['w1']}")
+    if shp["router_w"] != (dd, E):
+        raise ValueError(f"router_w must be {(dd, E)}, got {shp['router_w']}")
+    if len(shp["sl"]) == 2:
+        kb = 0
+        want = {"sl": (E, F), "sv": (E, F), "s1": (E, dd)}
+    else:
+        if len(shp["sl"]) != 3 or shp["sl"][1] == 0 or dd % shp["sl"][1]:
+            raise ValueError(f"sl must be [E, F] or [E, d/kb, F], got {shp['sl']}")
+        kb = dd // shp["sl"][1]
+        if F % kb:
+            raise ValueError(f"scale block {kb} does not divide F = {F}")
+        want = {"sl": (E, dd // kb, F), "sv": (E, dd // kb, F), "s1": (E, F // kb, dd)}
+    for k, v in want.items():
+        if shp[k] != v:
+            raise ValueError(f"{k} must be {v}, got {shp[k]}")
+    return E, dd, F, kb
+
+
 def scale_block(layer) -> int:
     """Block of inputs sharing a scale: 0 when the scales are per output channel ([E, out]),
     else in / (number of scale rows) for per-block scales ([E, in/kb, out])."""
@@ -189,6 +224,7 @@ def expert_ffn(xt: np.ndarray, layer, e: int, nthreads: int = 0, gelu_kind: int 
                return_h: bool = False):
     """One expert's gated-GELU FFN on one fp64 token row."""
     xt = np.ascontiguousarray(xt, dtype=np.float64)
+    check_layer(layer, xt.shape[0])
     wl, sl = _np(layer["wl"], np.int8), _np(layer["sl"], np.uint16)
     wv, sv = _np(layer["wv"], np.int8), _np(layer["sv"], np.uint16)
     w1, s1 = _np(layer["w1"], np.int8), _np(layer["s1"], np.uint16)
@@ -210,6 +246,7 @@ def forward(layer, x, bias=None, tokens: Optional[Sequence[int]] = None, forced_
     (out row 0, experts -1, gates 0)."""
     xb = _np(x, np.uint16)
     T, d = xb.shape
+    check_layer(layer, d)
     rw = _np(layer["router_w"], np.float32)
     wl, sl = _np(layer["wl"], np.int8), _np(layer["sl"], np.uint16)
     wv, sv = _np(layer["wv"], np.int8), _np(layer["sv"], np.uint16)
@@ -261,7 +298,9 @@ def block_chain(layers: List[dict], gammas: List[dict], h, eps: float = 1e-5,
     Per block b:  u = bf16( RMSNorm(h; g_pre) )        (the MoE layer's bf16 input)
                   y = MoE_b(u)                          (fp64)
                   h = bf16( h + RMSNorm(y; g_post) )    (bf16 residual stream)
-    Returns a list of per-block dicts: h_in (fp64 values of bf16), u, idx, gate, probs, h_out.
+    Returns a list of per-block dicts: h_in (fp64 values of bf16), u_exact (RMSNorm(h; g_pre)
+    before its bf16 rounding), u, idx, gate, probs, y, delta (RMSNorm(y; g_post), the fp64
+    value added to the residual stream before its bf16 rounding) and h_out.
     ``forced[b]`` (optional [n,2]) names the experts to use in block b.
     ``mask`` (optional [T]) marks padding tokens (0): their MoE output is 0, so their row of
     the residual stream passes through unchanged.
@@ -273,13 +312,16 @@ def block_chain(layers: List[dict], gammas: List[dict], h, eps: float = 1e-5,
     mk = None if mask is None else np.asarray(_np(mask)).astype(np.uint8).reshape(-1)[rows]
     res = []
     for b, (layer, gm) in enumerate(zip(layers, gammas)):
-        u = round_bf16(rmsnorm(cur, gm["pre"], eps))
+        u_exact = rmsnorm(cur, gm["pre"], eps)
+        u = round_bf16(u_exact)
         ub = f64_to_bf16_bits(u)
         r = route(ub, layer["router_w"])
         fb = None if forced is None else forced[b]
         y, idx, gate = forward(layer, ub, tokens=None, forced_idx=fb, nthreads=nthreads,
                                gelu_kind=gelu_kind, mask=mk)
-        nxt = round_bf16(cur + rmsnorm(y, gm["post"], eps))
-        res.append(dict(h_in=cur, u=u, idx=idx, gate=gate, probs=r["probs"], h_out=nxt))
+        delta = rmsnorm(y, gm["post"], eps)
+        nxt = round_bf16(cur + delta)
+        res.append(dict(h_in=cur, u_exact=u_exact, u=u, idx=idx, gate=gate, probs=r["probs"], y=y,
+                        delta=delta, h_out=nxt))
         cur = nxt
     return res

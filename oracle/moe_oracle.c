@@ -28,7 +28,7 @@
  *             residual h += h_dense) and the grok-field-guide source-code map,
  *             fourth stop (moe(rms_norm(h)) added to h).
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - the gate is the full 8-way softmax probability of the chosen expert; the
  *     two gates are not renormalised (the pages name no such step);
  *   - slot 0 holds the larger probability; equal logits go to the lower index;

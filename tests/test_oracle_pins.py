@@ -104,6 +104,16 @@ def test_gelu_tanh_form():
     assert abs(oracle.gelu(1e-6, 0) / 1e-6 - 0.5) < 1e-6
 
 
+def test_gelu_tanh_form_is_torch_tanh_gelu():
+    """The oracle's default GELU is torch's tanh-approximate GELU (a library routine written
+    independently of the oracle's C): a wrong 0.044715 or sqrt(2/pi) fails here."""
+    xs = torch.linspace(-9, 9, 4001, dtype=torch.float64)
+    xs = torch.cat([xs, torch.tensor([-1e-3, 1e-3, 0.3, -2.7, 5.5, 1e-8], dtype=torch.float64)])
+    ref = torch.nn.functional.gelu(xs, approximate="tanh").numpy()
+    got = np.array([oracle.gelu(float(x), 0) for x in xs])
+    assert np.max(np.abs(got - ref)) <= 1e-15 * np.maximum(1.0, np.abs(ref)).max()
+
+
 def test_gelu_erf_form_is_erf():
     for x in (-3.0, -0.7, 0.1, 1.0, 2.5):
         assert oracle.gelu(x, 1) == pytest.approx(0.5 * x * (1 + math.erf(x / math.sqrt(2))), rel=1e-15)
@@ -196,6 +206,42 @@ def test_expert_ffn_matches_numpy(tiny):
         y = oracle.expert_ffn(x64[t], layer, e, gelu_kind=1)
         ref = _dense_ffn(npl, e, x64[t])
         assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_expert_ffn_tanh_gelu_matches_numpy(tiny):
+    """The default (tanh) GELU branch of the expert FFN against numpy float64 matmuls with
+    torch's tanh-approximate GELU."""
+    layer = tiny.layers[0]
+    npl = _np_layer(layer)
+    x64 = tiny.x.to(torch.float64).numpy()
+    tanh_gelu = lambda a: torch.nn.functional.gelu(torch.from_numpy(a), approximate="tanh").numpy()
+    for e, t in [(1, 2), (6, 33)]:
+        y = oracle.expert_ffn(x64[t], layer, e)          # gelu_kind 0: the tanh form
+        ref = (tanh_gelu(x64[t] @ npl["Wl"][e]) * (x64[t] @ npl["Wv"][e])) @ npl["W1"][e]
+        assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_forward_rejects_inconsistent_shapes(tiny):
+    """A layer whose weights were transposed to another layout (or whose scales belong to
+    another matrix) is refused instead of being read as a layer of another width."""
+    layer = tiny.layers[0]
+    packed = dict(layer)
+    packed["wl"] = layer["wl"].transpose(1, 2).contiguous()
+    packed["wv"] = layer["wv"].transpose(1, 2).contiguous()
+    packed["w1"] = layer["w1"].transpose(1, 2).contiguous()
+    with pytest.raises(ValueError):
+        oracle.forward(packed, tiny.x, tokens=[0])
+    with pytest.raises(ValueError):
+        oracle.expert_ffn(tiny.x[0].to(torch.float64).numpy(), packed, 0)
+    swapped = dict(layer)
+    swapped["s1"] = layer["sl"]
+    with pytest.raises(ValueError):
+        oracle.forward(swapped, tiny.x, tokens=[0])
+    wrong_router = dict(layer)
+    wrong_router["router_w"] = layer["router_w"].t().contiguous()
+    with pytest.raises(ValueError):
+        oracle.forward(wrong_router, tiny.x, tokens=[0])
+    assert oracle.check_layer(layer, 256) == (8, 256, 512, 0)
 
 
 def test_forced_expert_reduces_to_dense_ffn(tiny):
@@ -348,6 +394,95 @@ def test_rmsnorm_properties():
     assert np.allclose(oracle.rmsnorm(z, gamma, eps=0.0), 2 * y, rtol=1e-14)
     # eps enters inside the root: a zero row stays zero, a tiny row is damped
     assert np.all(oracle.rmsnorm(np.zeros((1, 256)), None, eps=1e-5) == 0)
+
+
+def test_rmsnorm_constant_row_closed_form():
+    """A constant row c normalises to c / sqrt(c^2 + eps) (times the gain): this fixes where
+    eps enters (inside the root, added to the mean square).  With c = 1e-3 and eps = 1e-5
+    the reading c / (|c| + eps) would give 0.99 instead of 0.3015."""
+    d = 256
+    gamma = torch.full((d,), 1.5, dtype=torch.bfloat16)
+    for c, eps in ((1e-3, 1e-5), (0.25, 1e-5), (-3.0, 0.5), (2.0, 0.0)):
+        z = np.full((2, d), c)
+        got = oracle.rmsnorm(z, None, eps=eps)
+        want = c / math.sqrt(c * c + eps)
+        np.testing.assert_allclose(got, want, rtol=1e-15, atol=0)
+        np.testing.assert_allclose(oracle.rmsnorm(z, gamma, eps=eps), 1.5 * want, rtol=1e-15, atol=0)
+
+
+def _stack(seed=3, T=6):
+    w = moe_synth.Workload("tiny_stack", T=T, d=256, F=512, blocks=1, seed=seed)
+    inp = moe_synth.make_inputs(w, device="cpu")
+    g = torch.Generator().manual_seed(seed + 50)
+    # non-unit, non-uniform gains, so that a gain applied before its norm changes the result
+    gam = [{k: (0.5 + torch.rand(256, generator=g)).to(torch.bfloat16) for k in ("pre", "post")}]
+    return inp, gam
+
+
+def _times2(t):
+    return (t.to(torch.float32) * 2).to(t.dtype)   # exact in bf16 (power of two)
+
+
+def test_block_chain_pre_norm_is_applied():
+    """Scaling the residual stream by 2 leaves u = bf16(RMSNorm(h) * g_pre) and the routing
+    unchanged bit for bit when eps = 0; a chain that skipped the pre-norm would route 2h."""
+    inp, gam = _stack()
+    a = oracle.block_chain(inp.layers, gam, inp.x, eps=0.0)[0]
+    b = oracle.block_chain(inp.layers, gam, _times2(inp.x), eps=0.0)[0]
+    assert np.array_equal(a["u"], b["u"])
+    assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["gate"], b["gate"])
+    assert np.array_equal(a["delta"], b["delta"])
+    assert not np.array_equal(a["u"], a["h_in"])
+
+
+def test_block_chain_pre_gain_after_the_norm():
+    """Doubling g_pre doubles u exactly (the gain multiplies the normalised row); a gain
+    applied before the norm would cancel out and leave u unchanged."""
+    inp, gam = _stack()
+    a = oracle.block_chain(inp.layers, gam, inp.x, eps=1e-5)[0]
+    gam2 = [{"pre": _times2(gam[0]["pre"]), "post": gam[0]["post"]}]
+    b = oracle.block_chain(inp.layers, gam2, inp.x, eps=1e-5)[0]
+    assert np.array_equal(b["u"], 2 * a["u"])
+
+
+def test_block_chain_post_norm_is_applied():
+    """Scaling every linear_1 scale by 2 doubles the MoE output y exactly, and with eps = 0
+    the post-norm cancels it: the block's contribution and h_out are unchanged bit for bit.
+    A chain without the post-norm would add 2y instead of y."""
+    inp, gam = _stack()
+    a = oracle.block_chain(inp.layers, gam, inp.x, eps=0.0)[0]
+    layer2 = dict(inp.layers[0])
+    layer2["s1"] = _times2(layer2["s1"])
+    b = oracle.block_chain([layer2], gam, inp.x, eps=0.0)[0]
+    assert np.array_equal(b["y"], 2 * a["y"])
+    assert np.array_equal(b["delta"], a["delta"])
+    assert np.array_equal(b["h_out"], a["h_out"])
+
+
+def test_block_chain_post_gain_after_the_norm():
+    """Doubling g_post doubles the contribution exactly; a gain applied before the post-norm
+    would cancel out."""
+    inp, gam = _stack()
+    a = oracle.block_chain(inp.layers, gam, inp.x, eps=1e-5)[0]
+    gam2 = [{"pre": gam[0]["pre"], "post": _times2(gam[0]["post"])}]
+    b = oracle.block_chain(inp.layers, gam2, inp.x, eps=1e-5)[0]
+    assert np.array_equal(b["delta"], 2 * a["delta"])
+    assert not np.array_equal(b["h_out"], a["h_out"])
+
+
+def test_block_chain_residual_add():
+    """linear_1 scales 0: y = 0, RMSNorm(0) = 0 (eps > 0), so h_out equals h_in exactly; a
+    chain that dropped the residual add would return 0.  With real scales, h_out is the
+    bf16 rounding of h_in + delta."""
+    inp, gam = _stack()
+    layer0 = dict(inp.layers[0])
+    layer0["s1"] = torch.zeros_like(layer0["s1"])
+    z = oracle.block_chain([layer0], gam, inp.x, eps=1e-5)[0]
+    assert np.all(z["y"] == 0) and np.all(z["delta"] == 0)
+    assert np.array_equal(z["h_out"], z["h_in"])
+    a = oracle.block_chain(inp.layers, gam, inp.x, eps=1e-5)[0]
+    assert np.array_equal(a["h_out"], torch.from_numpy(a["h_in"] + a["delta"]).to(torch.bfloat16)
+                          .to(torch.float64).numpy())
 
 
 def test_block_chain_rows_are_independent(tiny):
