@@ -3,27 +3,35 @@
 shape (d_model 6144, ffn 32768, 8 experts, top-2, int8 weights) and the fraction
 of the HBM / bf16 tensor roofline reached by the dominant kernel.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|stacked]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed|stacked]
     python bench.py --impl reference ...      # the fp64 CPU oracle on the host cores
 
 One step = one pass of the whole layer (router, dispatch, gather, up-projection,
 down-projection, combine) over one batch of T synthetic tokens; the stacked
-workload's step is its four residual blocks.  Inputs are resident in HBM when
-the timed region starts; the layer weights (4.8 GB) are larger than L2, so every
-step streams them from HBM.  Under torchrun each rank runs an independent
-replica on its own GPU and its own token batch (no collective on the data path);
-the reported value is all ranks' tokens over the slowest rank's time.
+workload's step is its four residual blocks.  The headline line is the prefill
+workload (T = 8192, one full context: the largest configuration, bound by the bf16
+tensor pipe); with no --workload it also carries a `workloads` object with the
+decode (HBM-bound), skewed-routing and stacked-block workloads and the API weight
+layout's decode and prefill, each measured the same way.
+
+Timing: W untimed warm-up steps, then R repeats of a region of exactly K steps,
+each bracketed by a barrier and a device synchronisation and timed with CUDA events
+on the launching stream; the reported time is the median region.  Inputs are
+resident in HBM when a region starts; the layer weights (4.8 GB per layer) are
+larger than L2, so every step streams them from HBM.  Under torchrun each rank runs
+an independent replica on its own GPU and its own token batch (no collective on the
+data path); the reported value is all ranks' tokens over the slowest rank's time.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
 import sys
-import tempfile
 import threading
 import time
 
@@ -32,17 +40,26 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/sec at Grok-1 shape; % of HBM / bf16 tensor-pipe roofline"
 KERNELS = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine", "prenorm", "route_small")
+DATA = "synthetic (seeded; random-init int8 weights of the Grok-1 MoE shape)"
+
+# sub-records of the default run: (record name, workload, weight layout)
+SUBRECORDS = (("decode", "decode", "packed"), ("skewed", "skewed", "packed"), ("stacked", "stacked", "packed"),
+              ("decode_api_layout", "decode", "in_out"), ("prefill_api_layout", "prefill", "in_out"))
+TIMED_SECONDS = 1.5       # repeats of the K-step region fill about this much device time
+SUB_CPU_SECONDS = 5.0     # oracle budget of each sub-record's CPU baseline
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=None)
     p.add_argument("--warmup", type=int, default=None)
     p.add_argument("--impl", choices=("native", "reference"), default="native")
-    p.add_argument("--workload", default="decode", choices=("decode", "prefill", "skewed", "stacked", "tiny"))
+    p.add_argument("--workload", default=None, choices=("decode", "prefill", "skewed", "stacked", "tiny"),
+                   help="one workload only (default: prefill as the headline plus the sub-records)")
+    p.add_argument("--repeats", type=int, default=None, help="timed K-step regions (default: ~1.5 s of them)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the headline's oracle sample")
     # smaller variants of a workload for profiler captures (never a bench line)
     p.add_argument("--tokens", type=int, default=None, help="override T")
     p.add_argument("--ffn", type=int, default=None, help="override the FFN width")
@@ -51,13 +68,21 @@ def parse():
                    help="weight scale format: 0 per output channel, 128 per block of 128 inputs (packed layout)")
     p.add_argument("--layout", choices=("packed", "in_out"), default="packed",
                    help="weight layout: packed = tiles written once at load (TMEM path); in_out = as drawn")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 def default_steps(workload):
-    # enough steps that the timed region lasts about a second or more
-    return {"decode": (1000, 20), "stacked": (300, 10), "prefill": (40, 5), "skewed": (60, 5),
-            "tiny": (1000, 20)}[workload]
+    return {"decode": (200, 10), "stacked": (50, 5), "prefill": (20, 5), "skewed": (20, 5),
+            "tiny": (200, 10)}[workload]
+
+
+def repeats_for(ms_per_step: float, steps: int, requested=None) -> int:
+    """Timed regions of `steps` steps: enough to fill about TIMED_SECONDS (so that the clock
+    sampler sees the timed regions themselves), at least 3, at most 200."""
+    if requested:
+        return max(1, int(requested))
+    region_s = max(ms_per_step, 1e-3) * steps / 1e3
+    return int(min(200, max(3, math.ceil(TIMED_SECONDS / region_s))))
 
 
 # ---- distributed plumbing --------------------------------------------------------
@@ -152,28 +177,34 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.th.join(timeout=2)
-        rows = []
-        for ts, line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
-            except ValueError:
-                continue
-        if not rows:
-            return None
-        inside = [r for r in rows if self.t0 and self.t1 and self.t0 <= r[0] <= self.t1]
-        use = inside if inside else rows
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = set()
-        for r in use:
-            for nm, v in zip(names, r[3][1:]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
-                "reasons": sorted(reasons), "samples": len(use),
-                "window": "timed region" if inside else "whole run (timed region shorter than one sample)"}
+        return summarize_clocks(self.lines, self.t0, self.t1)
+
+
+def summarize_clocks(lines, t0, t1):
+    """nvidia-smi rows (time, csv line) -> median SM clock, max clock and the throttle reasons
+    seen, over the rows inside [t0, t1] (all rows when none falls inside)."""
+    rows = []
+    for ts, line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
+        except ValueError:
+            continue
+    if not rows:
+        return None
+    inside = [r for r in rows if t0 and t1 and t0 <= r[0] <= t1]
+    use = inside if inside else rows
+    names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    reasons = set()
+    for r in use:
+        for nm, v in zip(names, r[3][1:]):
+            if v.lower() == "active":
+                reasons.add(nm)
+    return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+            "reasons": sorted(reasons), "samples": len(use),
+            "window": "timed region" if inside else "whole run (timed region shorter than one sample)"}
 
 
 # ---- roofline bookkeeping ----------------------------------------------------------
@@ -229,21 +260,44 @@ def algorithmic_work(w, T, n_touched, counts, kblock=0):
     return dict(up_bytes=up_bytes, dn_bytes=dn_bytes, up_flops=up_flops, dn_flops=dn_flops)
 
 
+def roofline_of(workload, layout, work, up_ms, peaks, peak_src, variant):
+    """The dominant kernel (the up-projection) against its bound: the sustained bf16 GEMM figure
+    for the tensor-bound workloads (its time comes from back-to-back steps under the power cap;
+    the burst fraction is context), measured copy bandwidth for the HBM-bound ones."""
+    if workload in ("prefill", "skewed"):
+        achieved = work["up_flops"] / (up_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "frac_of_burst": achieved / peaks["bf16_tflops"], "kernel": "up_proj",
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
+                "traffic": recorded_traffic(workload, layout, "up_proj", variant),
+                "algorithmic_flops_per_launch": work["up_flops"], "launch_ms": up_ms}
+    achieved = work["up_bytes"] / (up_ms / 1e3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "kernel": "up_proj", "peak_source": f"{peak_src} hbm_gbs (copy)",
+            "traffic": recorded_traffic(workload, layout, "up_proj", variant),
+            "algorithmic_bytes_per_launch": work["up_bytes"], "launch_ms": up_ms}
+
+
 # ---- the CUDA path -------------------------------------------------------------------
 
-def run_native(args, world, rank, local):
+def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
+    """One workload, measured: the K-step regions, the per-kernel pass, the end-to-end pass
+    with host buffers and (rank 0, one process) the oracle on the host cores.  Returns the
+    record and the number of this library's kernel launches per step."""
     import torch
     import moe_synth
     import mixture_experts_softmax_b200 as moe
 
-    w = moe_synth.WORKLOADS[args.workload]
+    w = moe_synth.WORKLOADS[name]
     if args.tokens or args.ffn:
         import dataclasses
         w = dataclasses.replace(w, T=args.tokens or w.T, F=args.ffn or w.F, name=w.name + "_resized")
     variant = bool(args.tokens or args.ffn or args.scale_block)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    K, W = args.steps, args.warmup
+    ks, ws = default_steps(name)
+    K = args.steps if args.steps is not None else ks
+    W = max(3, args.warmup if args.warmup is not None else ws)
     inp = moe_synth.make_inputs(w, device=dev, seed=w.seed)
     if world > 1:   # each replica gets its own token batch; the layer weights are the same model
         g = moe_synth.generator(w.seed + 1000 + rank, dev)
@@ -253,13 +307,14 @@ def run_native(args, world, rank, local):
     if args.scale_block:   # per-block scale format: the same weights, one scale row per 128 inputs
         gs = moe_synth.generator(w.seed + 2000, dev)
         layers = [moe_synth.block_scales(l, args.scale_block, gs) for l in layers]
-    bias = inp.bias
+    # the oracle reads the layer as drawn ([E, in, out]); keep host copies before any repacking
+    cpu_layers = [{k: v.cpu() for k, v in l.items()} for l in layers] if with_cpu else None
     stream = torch.cuda.current_stream(dev)
 
     h = moe.MoELayer(w.d, w.F, w.E, w.k)
-    moe.check(moe.moe_set_router_bias(h.h, bias))
+    moe.check(moe.moe_set_router_bias(h.h, inp.bias))
     moe.check(moe.moe_set_scale_block(h.h, args.scale_block))
-    if args.layout == "packed":
+    if layout == "packed":
         # one-time weight-load step, outside every timed region: K-major int8 copies
         moe.check(moe.moe_set_weight_layout(h.h, moe.MOE_LAYOUT_PACKED))
         drawn = layers
@@ -269,9 +324,11 @@ def run_native(args, world, rank, local):
             for k in ("wl", "wv", "w1"):
                 l[k] = None
         del drawn
+        inp.layers = None
         torch.cuda.empty_cache()
     out = torch.empty_like(inp.x)
     res0 = inp.x.clone()
+    hio = torch.empty_like(inp.x)
 
     def step():
         if w.blocks:
@@ -282,41 +339,59 @@ def run_native(args, world, rank, local):
         else:
             moe.check(moe.moe_forward(h.h, T, inp.x, *moe.layer_args(layers[0]), out, stream))
 
-    hio = torch.empty_like(inp.x)
+    # warm-up (timed only to size the repeats)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
     for _ in range(W):
         step()
+    e1.record(stream)
     moe.check(moe.moe_sync_status(h.h, stream))
+    R = repeats_for(e0.elapsed_time(e1) / W, K, args.repeats)
+    R = int(max_over_ranks(R, world, dev))   # every rank runs the same number of regions
 
-    # headline: K steps, device-timed
+    # R regions of exactly K steps, device-timed; the median region is reported
     clocks = ClockSampler(dev.index) if rank == 0 else None
     if clocks:
         clocks.start()
-    barrier(world, dev)
-    torch.cuda.synchronize(dev)
-    if clocks:
-        clocks.mark("t0")
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    region_ms = []
+    for r in range(R):
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        if clocks and r == 0:
+            clocks.mark("t0")
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        region_ms.append(e0.elapsed_time(e1))
     if clocks:
         clocks.mark("t1")
     barrier(world, dev)
-    ms = e0.elapsed_time(e1) / K
     clk = clocks.stop() if clocks else None
     moe.check(moe.moe_sync_status(h.h, stream), "device status after the timed region")
+    ms = statistics.median(region_ms) / K
     value, ms_max = job_value(T, world, ms, dev)
     tokens = T * world
+    rec = {"value": value, "unit": "tokens/s", "ms_per_step": ms_max, "steps": K, "warmup": W, "repeats": R,
+           "region_ms": {"min": min(region_ms), "median": statistics.median(region_ms), "max": max(region_ms)},
+           "config": {"workload": w.name, "T_per_gpu": T, "d_model": w.d, "ffn": w.F, "experts": w.E,
+                      "top_k": w.k, "blocks": w.blocks or 1,
+                      "router_bias": w.bias,
+                      "weights": "int8 + bf16 " + ("scales per block of %d inputs" % args.scale_block
+                                                   if args.scale_block else "per-output-channel scales") +
+                                 ", layout " + layout +
+                                 (" (packed once at load, untimed)" if layout == "packed" else " (as drawn)"),
+                      "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],
+                      "down_splits": moe.moe_plan(h.h, T)[2]},
+           "clocks": clk}
 
     if args.skip_extras:
         h.close()
-        return {"metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": ms_max, "n_gpus": world,
-                "steps": K, "warmup": W, "config": {"workload": w.name, "T_per_gpu": T, "ffn": w.F},
-                "note": "profiling variant: no per-kernel or end-to-end pass"}
+        rec["note"] = "profiling variant: no per-kernel or end-to-end pass"
+        return rec, None
 
-    # per-kernel durations: the same K steps again with events around every launch
+    # per-kernel durations: K more steps with events around every launch
     moe.check(moe.moe_set_profiling(h.h, True))
     moe.moe_get_kernel_times(h.h)
     barrier(world, dev)
@@ -336,48 +411,39 @@ def run_native(args, world, rank, local):
     counts = [off[e + 1] - off[e] for e in range(w.E)]
     n_touched = sum(1 for c in counts if c > 0)
 
-    # end to end through the host-buffer entry point (pinned host memory, copies timed)
-    e2e = None
-    if not w.blocks:
-        x_host = inp.x.cpu().pin_memory()
-        out_host = torch.empty_like(x_host).pin_memory()
-        for _ in range(max(1, W // 2)):
+    # end to end through the public API with host buffers: pinned input in, result out, every step
+    x_host = inp.x.cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    if w.blocks:
+        def e2e_step():   # the residual stream in, four blocks, the residual stream out
+            hio.copy_(x_host, non_blocking=True)
+            for b in range(w.blocks):
+                moe.check(moe.moe_block_forward(h.h, T, hio, inp.gammas[b]["pre"], inp.gammas[b]["post"], w.eps,
+                                                *moe.layer_args(layers[b]), stream))
+            out_host.copy_(hio, non_blocking=True)
+        api = "moe_block_forward x%d with pinned host copies of the residual stream" % w.blocks
+    else:
+        def e2e_step():
             moe.check(moe.moe_forward_host(h.h, T, x_host, *moe.layer_args(layers[0]), out_host, stream))
-        barrier(world, dev)
-        torch.cuda.synchronize(dev)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(K):
-            moe.check(moe.moe_forward_host(h.h, T, x_host, *moe.layer_args(layers[0]), out_host, stream))
-        f1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / K, world, dev)
-        moe.check(moe.moe_sync_status(h.h, stream))
-        nb = T * w.d * 2
-        e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": nb,
-               "d2h_bytes_per_step": nb, "ms_per_step": e2e_ms, "api": "moe_forward_host"}
+        api = "moe_forward_host"
+    for _ in range(max(1, W // 2)):
+        e2e_step()
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, world, dev)
+    moe.check(moe.moe_sync_status(h.h, stream))
+    nb = T * w.d * 2
+    rec["e2e"] = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": nb,
+                  "d2h_bytes_per_step": nb, "ms_per_step": e2e_ms, "api": api}
 
     peaks, peak_src = measured_peaks()
     work = algorithmic_work(w, T, n_touched, counts, args.scale_block)
-    up_ms = per_launch["up_proj"]
-    dn_ms = per_launch["down_proj"]
-    if args.workload in ("prefill", "skewed"):
-        # the per-kernel times come from K back-to-back steps (about a second of GEMMs under the
-        # power cap): the sustained GEMM figure is the denominator, the burst one is context
-        achieved = work["up_flops"] / (up_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "frac_of_burst": achieved / peaks["bf16_tflops"],
-                "kernel": "up_proj", "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
-                "traffic": recorded_traffic(args.workload, args.layout, "up_proj", variant),
-                "algorithmic_flops_per_launch": work["up_flops"], "launch_ms": up_ms}
-    else:
-        achieved = work["up_bytes"] / (up_ms / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "kernel": "up_proj", "peak_source": f"{peak_src} hbm_gbs (copy)",
-                "traffic": recorded_traffic(args.workload, args.layout, "up_proj", variant),
-                "algorithmic_bytes_per_launch": work["up_bytes"], "launch_ms": up_ms}
+    rec["roofline"] = roofline_of(name, layout, work, per_launch["up_proj"], peaks, peak_src, variant)
     layer_bytes = (work["up_bytes"] + work["dn_bytes"]) * (w.blocks or 1)
     layer_roof = {"bytes_per_step": layer_bytes, "GBps": layer_bytes / (ms / 1e3) / 1e9,
                   "frac_hbm": layer_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
@@ -385,43 +451,57 @@ def run_native(args, world, rank, local):
     layer_roof["TFLOPs"] = layer_roof["flops_per_step"] / (ms / 1e3) / 1e12
     layer_roof["frac_tensor"] = layer_roof["TFLOPs"] / peaks["bf16_tflops_sustained"]
     layer_roof["frac_tensor_of_burst"] = layer_roof["TFLOPs"] / peaks["bf16_tflops"]
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, layers, inp, args.cpu_seconds)
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded; random-init int8 weights of the Grok-1 MoE shape)",
-        "config": {"workload": args.workload, "T_per_gpu": T, "d_model": w.d, "ffn": w.F, "experts": w.E,
-                   "top_k": w.k, "blocks": w.blocks or 1,
-                   "weights": "int8 + bf16 " + ("scales per block of %d inputs" % args.scale_block
-                                                if args.scale_block else "per-output-channel scales") +
-                              ", layout " + args.layout +
-                              (" (packed once at load, untimed)" if args.layout == "packed" else ""),
-                   "l2": "inputs larger than L2 (%.2f GB of weights per step)" % (layer_bytes / 1e9),
-                   "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],
-                   "down_splits": moe.moe_plan(h.h, T)[2]},
-        "roofline": roof,
-        "layer": layer_roof,
-        "kernel_ms": per_launch,
-        "experts_touched": n_touched,
-        "gpu_launches": int(round(launches_per_step * K)),
-        "e2e": e2e,
-        "clocks": clk,
-        "cpu_baseline": cpu,
-    }
+    dn_ms = per_launch["down_proj"]
+    layer_roof["down_proj"] = ({"GBps": work["dn_bytes"] / (dn_ms / 1e3) / 1e9,
+                                "frac_hbm": work["dn_bytes"] / (dn_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                                "TFLOPs": work["dn_flops"] / (dn_ms / 1e3) / 1e12,
+                                "frac_tensor": work["dn_flops"] / (dn_ms / 1e3) / 1e12 /
+                                peaks["bf16_tflops_sustained"]} if dn_ms > 0 else None)
+    rec["layer"] = layer_roof
+    rec["kernel_ms"] = per_launch
+    rec["experts_touched"] = n_touched
+    rec["config"]["l2"] = "inputs larger than L2 (%.2f GB of weights per step)" % (layer_bytes / 1e9)
+    rec["cpu_baseline"] = cpu_baseline(w, cpu_layers, inp, cpu_seconds) if with_cpu else None
     h.close()
+    return rec, launches_per_step
+
+
+def run_native(args, world, rank, local):
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    head = args.workload or "prefill"
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    rec, lps = bench_workload(head, args, world, rank, dev, args.layout, args.cpu_seconds, with_cpu)
+    line = {"metric": METRIC, "value": rec["value"], "unit": "tokens/s", "n_gpus": world, "steps": rec["steps"],
+            "warmup": rec["warmup"], "repeats": rec["repeats"], "ms_per_step": rec["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA}
+    line.update({k: v for k, v in rec.items() if k not in line and k not in ("unit",)})
+    if lps is not None:
+        line["gpu_launches"] = int(round(lps * rec["steps"]))
+        line["gpu_launches_note"] = ("this library's kernel launches in one timed region of %d steps (%g per step; "
+                                     "%d such regions were timed)" % (rec["steps"], lps, rec["repeats"]))
+    # the other workloads, one process only (a multi-GPU run reports the headline workload)
+    if args.workload is None and world == 1 and not (args.tokens or args.ffn):
+        subs = {}
+        for key, wname, layout in SUBRECORDS:
+            import gc
+            gc.collect()
+            torch.cuda.empty_cache()
+            # the API layout computes the same layer: its oracle baseline is the packed record's
+            sub, slps = bench_workload(wname, argparse.Namespace(**{**vars(args), "steps": None, "warmup": None}),
+                                       world, rank, dev, layout, SUB_CPU_SECONDS, with_cpu and layout == "packed")
+            if slps is not None:
+                sub["gpu_launches_per_step"] = slps
+            subs[key] = sub
+        line["workloads"] = subs
     return line
 
 
-def cpu_baseline(w, layers, inp, budget_s):
-    """The fp64 oracle on the host cores on a bounded sample of the same workload."""
-    import numpy as np
-    import torch
+def cpu_baseline(w, cpu_layers, inp, budget_s):
+    """The fp64 oracle on the host cores on a bounded sample of the same workload: the routing
+    of the whole batch, then the expert FFNs of as many tokens as fit in the budget."""
     import oracle
-    cpu_layers = [{k: v.cpu() for k, v in l.items()} for l in layers]
     x = inp.x.cpu()
     cores = os.cpu_count()
     t_start = time.time()
@@ -447,10 +527,10 @@ def cpu_baseline(w, layers, inp, budget_s):
 # ---- the reference arm: the CPU oracle ------------------------------------------------
 
 def run_reference(args, world, rank):
-    import torch
     import moe_synth
     import oracle
-    w = moe_synth.WORKLOADS[args.workload]
+    name = args.workload or "prefill"
+    w = moe_synth.WORKLOADS[name]
     inp = moe_synth.make_inputs(w, device="cpu")
     K, W = args.steps, args.warmup
     x = inp.x
@@ -477,8 +557,8 @@ def run_reference(args, world, rank):
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": dt / K * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; random-init int8 weights of the Grok-1 MoE shape)",
-        "config": {"workload": args.workload, "T_per_gpu": w.T, "d_model": w.d, "ffn": w.F, "experts": w.E,
+        "vs_baseline": None, "dtype": "f64", "data": DATA,
+        "config": {"workload": name, "T_per_gpu": w.T, "d_model": w.d, "ffn": w.F, "experts": w.E,
                    "top_k": w.k, "blocks": w.blocks or 1},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -487,28 +567,21 @@ def run_reference(args, world, rank):
 
 def main():
     args = parse()
-    ks, ws = default_steps(args.workload)
-    if args.steps is None:
-        args.steps = ks
-    if args.warmup is None:
-        args.warmup = ws
-    if args.warmup < 3:
-        args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         if rank != 0:
             return 0
+        ks, ws = default_steps(args.workload or "prefill")
+        args.steps = ks if args.steps is None else args.steps
+        args.warmup = max(3, ws if args.warmup is None else args.warmup)
         if args.steps > 50 and args.workload != "tiny":
             args.steps = 20    # each step is about a second of fp64 work on the host
         line = run_reference(args, world, rank)
         print(json.dumps(line), flush=True)
         return 0
     world, rank, local = dist_setup(args.gpus)
-    try:
-        line = run_native(args, world, rank, local)
-    finally:
-        pass
+    line = run_native(args, world, rank, local)
     if rank == 0:
         print(json.dumps(line), flush=True)
     dist_teardown(world)

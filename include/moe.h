@@ -19,8 +19,10 @@
  *     tensor dense and row-major with the layout stated below.
  *   - bf16 tensors are passed as void* (IEEE bfloat16, 2 bytes per element).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *     Calls only enqueue work on it: none synchronises the host except
- *     moe_sync_status and moe_get_kernel_times, which say so.
+ *     Calls only enqueue work on it.  The host waits only in moe_sync_status,
+ *     moe_get_kernel_times and moe_destroy, and in a forward call that has to
+ *     grow the handle's workspace or that follows a call of the same handle on
+ *     another stream (it then first synchronises that earlier stream).
  *   - Every call returns MOE_OK (0) or a negative MOE_E* code; no exception or
  *     abort crosses the ABI.  Arguments are checked on the host before any CUDA
  *     call, so an invalid call has no effect on the device.
@@ -81,9 +83,13 @@ MOE_API int moe_version(void);
  * width from widening_factor, num_experts, num_selected_experts).
  * Supported: E == 8, k == 2, d % 128 == 0, ffn % 128 == 0, 128 <= d, ffn <= 65536.
  * Returns MOE_EINVAL for non-positive sizes or k > E, MOE_EUNSUPPORTED for
- * other shapes.  Allocates host memory only; device memory is taken on the
- * first forward call (stream-ordered) and grows with the largest T seen.
- * On success *out owns the handle; release it with moe_destroy.
+ * other shapes.  Allocates host memory only.  Device memory (the workspace) is
+ * taken with cudaMalloc on the first forward call and grows with the largest T
+ * seen: a forward call that has to grow it first synchronises the stream of the
+ * handle's previous call and frees the smaller buffers, so that call blocks the
+ * host until the earlier work is done.  Forwards that fit the workspace allocate
+ * nothing and do not block.  On success *out owns the handle; release it with
+ * moe_destroy.
  */
 MOE_API int moe_create(int d, int ffn, int E, int k, moe_handle *out);
 
@@ -162,7 +168,10 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
  * One residual MoE block ("Transformer stack and language model head": pre/post
  * RMSNorm around the MoE, h += h_dense), in place on the residual stream:
  *   u = bf16( RMSNorm(h; g_pre) ),   h <- bf16( h + RMSNorm( MoE(u); g_post ) )
- * with RMSNorm(z; g) = z / sqrt(mean(z^2) + eps) * g evaluated in fp32.
+ * with RMSNorm(z; g) = z / sqrt(mean(z^2) + eps) * g evaluated in fp32.  The
+ * routing kernels form u as they read h (no separate normalisation pass) and the
+ * post-norm and residual add run inside the combine; u stays in the handle's
+ * workspace until the next forward (moe_get_block_input).
  *   h_io          bf16 [T, d]  residual stream, read and overwritten
  *   g_pre, g_post bf16 [d]     RMSNorm gains
  * Other arguments as in moe_forward.
@@ -182,6 +191,16 @@ MOE_API int moe_block_forward(moe_handle h, int T, void *h_io, const void *g_pre
  */
 MOE_API int moe_get_routing(moe_handle h, int32_t *idx, float *gate, int32_t *offsets,
                             int32_t *perm, void *stream);
+
+/*
+ * Copy the bf16 MoE input u = bf16(RMSNorm(h; g_pre)) of the handle's last forward
+ * (device to device, on `stream`) into u: bf16 [T, d], 16-byte aligned.  This is
+ * the row the layer routed and multiplied, so a test can check the routing and the
+ * expert outputs on the very values the kernels used.  Returns MOE_EINVAL if the
+ * last forward was not moe_block_forward (or none ran), MOE_ECUDA if the copy
+ * could not be enqueued.
+ */
+MOE_API int moe_get_block_input(moe_handle h, void *u, void *stream);
 
 /*
  * Synchronise `stream`, then report the device status of the handle's kernels:
@@ -204,7 +223,8 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns);
  * moe_set_profiling(h, 1) starts recording around each kernel of every forward;
  * moe_get_kernel_times synchronises on those events and returns, per kernel id
  * (0 router, 1 dispatch, 2 gather, 3 up-projection, 4 down-projection,
- * 5 combine, 6 pre-norm, 7 small-batch routing: router and dispatch in one
+ * 5 combine, 6 unused (the residual block's pre-norm runs inside the routing
+ * kernels), 7 small-batch routing: router and dispatch in one
  * launch, used instead of 0-2 when T <= 32; in MOE_LAYOUT_PACKED the
  * up-projection then loads the routed rows itself, in MOE_LAYOUT_IN_OUT that
  * launch also gathers them), the total milliseconds and the
@@ -261,8 +281,9 @@ MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits);
  * Scratch: dispatch's working arrays live in one file-scope device array of about
  * 1 MB (MOE_NOALLOC_MAX_TOKENS tokens), which every GPU that loads the library holds
  * until the process exits.  The first call on a device looks up that array's device
- * address (cudaGetSymbolAddress, with the device current); make that first call
- * before any stream capture.  Every call shares the array and it keeps the last
+ * address (cudaGetSymbolAddress, with the device current) and keeps it while the same
+ * CUDA context stays current (a new context, e.g. after cudaDeviceReset, looks it up
+ * again); make that first call before any stream capture.  Every call shares the array and it keeps the last
  * call's contents; each call writes every word it later reads, so nothing needs
  * clearing, but calls whose kernels overlap on the GPU (different streams, or
  * concurrent host threads) race on it: serialise them.

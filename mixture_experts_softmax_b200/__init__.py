@@ -37,7 +37,7 @@ KERNEL_NAMES = ("router", "dispatch", "gather", "up_proj", "down_proj", "combine
 EXPORTS = (
     "moe_strerror", "moe_version", "moe_create", "moe_destroy", "moe_set_router_bias", "moe_set_padding_mask",
     "moe_set_scale_block",
-    "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing",
+    "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing", "moe_get_block_input",
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
     "moe_set_weight_layout", "moe_pack_weight", "moe_route_noalloc",
 )
@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "moe_forward_host": (I, [P, I, P, P, P, P, P, P, P, P, P, P]),
         "moe_block_forward": (I, [P, I, P, P, P, F, P, P, P, P, P, P, P, P]),
         "moe_get_routing": (I, [P, P, P, P, P, P]),
+        "moe_get_block_input": (I, [P, P, P]),
         "moe_sync_status": (I, [P, P]),
         "moe_set_timeout": (I, [P, ctypes.c_longlong]),
         "moe_set_profiling": (I, [P, I]),
@@ -167,6 +168,11 @@ def moe_block_forward(h, T, h_io, g_pre, g_post, eps, router_w, w_lin, s_lin, w_
 
 def moe_get_routing(h, idx=None, gate=None, offsets=None, perm=None, stream=None) -> int:
     return _lib.moe_get_routing(h, _ptr(idx), _ptr(gate), _ptr(offsets), _ptr(perm), _stream(stream))
+
+
+def moe_get_block_input(h, u, stream=None) -> int:
+    """u: device bf16 [T, d] receiving the last moe_block_forward's MoE input."""
+    return _lib.moe_get_block_input(h, _ptr(u), _stream(stream))
 
 
 def moe_sync_status(h, stream=None) -> int:

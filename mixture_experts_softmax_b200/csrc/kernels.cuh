@@ -25,8 +25,8 @@ struct RouteArgs {
     const float *bias;          // [E] or nullptr
     int *idx;                   // [T, 2]
     float *gate;                // [T, 2]
-    // optional pre-MoE RMSNorm (small-batch routing only): route on u = bf16(x * rsqrt(mean x^2 + eps) * g),
-    // written to u for the gather
+    // optional pre-MoE RMSNorm of the residual block: route on u = bf16(x * rsqrt(mean x^2 + eps) * g),
+    // written to u for the gather (every routing kernel)
     const __nv_bfloat16 *g_pre; // [d] or nullptr
     float eps;
     __nv_bfloat16 *u;           // [T, d]
@@ -96,13 +96,6 @@ struct CombineArgs {
     float eps;
 };
 
-struct NormArgs {
-    int T, d;
-    const __nv_bfloat16 *h;     // [T, d]
-    const __nv_bfloat16 *g;     // [d]
-    float eps;
-    __nv_bfloat16 *u;           // [T, d]
-};
 
 cudaError_t launch_router(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
@@ -130,7 +123,6 @@ int gemm_ts_kstage(bool up, int bn);
 // out[e, m, k] = in[e, k, m] for E int8 [K, M] matrices (K, M multiples of 64)
 cudaError_t launch_transpose_i8(const int8_t *in, int8_t *out, int E, int K, int M, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
-cudaError_t launch_prenorm(const NormArgs &a, cudaStream_t s);
 
 // dynamic shared memory each GEMM variant needs (for cudaFuncSetAttribute)
 size_t gemm_smem_bytes(bool up, int bn);

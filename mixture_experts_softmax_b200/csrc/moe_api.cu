@@ -57,6 +57,7 @@ struct moe_ctx {
     int route_cap = 0;      // T the route buffer holds
     int map_gen = 0;        // bumps when b_xp / b_h move
     int last_T = -1;
+    int last_block_T = -1;  // T of the last forward if it was moe_block_forward (u is staged), else -1
 
     // TMA descriptors
     std::vector<WeightMap> wmaps;
@@ -391,19 +392,14 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     if ((rc = weight_map(h, w_1, 1, &m_w1)) != MOE_OK) return rc;
     if ((rc = act_maps(h, bn, &m_xp, &m_h)) != MOE_OK) return rc;
 
-    // residual block: the routed rows are u = pre-RMSNorm(x), in the staging buffer; small
-    // batches normalise inside the routing launch, larger ones in a pre-norm launch first
+    // residual block: the routed rows are u = pre-RMSNorm(x); the routing kernels normalise
+    // each row as they read it and leave u in the staging buffer for the gather
     const bool small = T <= route_small_max_tokens();
     __nv_bfloat16 *u = static_cast<__nv_bfloat16 *>(h->b_stage.ptr);
     const __nv_bfloat16 *routed = static_cast<const __nv_bfloat16 *>(x);
-    if (g_pre && !small) {
-        NormArgs na{T, h->d, routed, static_cast<const __nv_bfloat16 *>(g_pre), eps, u};
-        if (timed(h, K_PRENORM, s, [&] { return launch_prenorm(na, s); }) != cudaSuccess) return MOE_ECUDA;
-        routed = u;
-    }
     RouteArgs ra{T, h->d, routed, router_w, h->bias, idx, gate};
     ra.mask = h->mask;
-    if (g_pre && small) {
+    if (g_pre) {
         ra.g_pre = static_cast<const __nv_bfloat16 *>(g_pre);
         ra.eps = eps;
         ra.u = u;
@@ -479,6 +475,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
         }) != cudaSuccess)
         return MOE_ECUDA;
 
+    h->last_block_T = g_pre ? T : -1;
     CombineArgs ca{T, h->d, splits, static_cast<const float *>(h->b_slots.ptr), idx, static_cast<__nv_bfloat16 *>(out),
                    static_cast<__nv_bfloat16 *>(h_io), static_cast<const __nv_bfloat16 *>(g_post), eps};
     if (timed(h, K_COMBINE, s, [&] { return launch_combine(ca, s); }) != cudaSuccess) return MOE_ECUDA;
@@ -688,6 +685,16 @@ MOE_API int moe_get_routing(moe_handle h, int32_t *idx, float *gate, int32_t *of
         if (c.dst && cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
             return MOE_ECUDA;
     return MOE_OK;
+}
+
+MOE_API int moe_get_block_input(moe_handle h, void *u, void *stream)
+{
+    if (!h || !u || !aligned16(u) || h->last_block_T < 0) return MOE_EINVAL;
+    const size_t bytes = static_cast<size_t>(h->last_block_T) * h->d * 2;
+    return cudaMemcpyAsync(u, h->b_stage.ptr, bytes, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ECUDA;
 }
 
 MOE_API int moe_sync_status(moe_handle h, void *stream)

@@ -7,6 +7,8 @@
 // without any allocation: the caller passes the inputs and the outputs, and the
 // dispatch step's own working arrays live in one file-scope device array that every
 // GPU loading this library holds until the process exits.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "../../include/moe.h"
@@ -32,10 +34,32 @@ static __device__ __align__(256) int g_route_scratch[kScratchWords];
 namespace {
 
 std::mutex g_mu;
-int *g_scratch_dev[64];   // device address of g_route_scratch, per CUDA device (set up once each)
+// device address of g_route_scratch per CUDA device, with the context it was looked up in:
+// the module (and so the array) is loaded again in a new context, for instance after
+// cudaDeviceReset, so an address is reused only while the same context is current
+int *g_scratch_dev[64];
+CUcontext g_scratch_ctx[64];
 
-// Device address of the scratch on the current device.  Done once per device with that
-// device current: in host code the array's name is only a host-side stand-in.
+CUcontext current_context()
+{
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    }
+    CUcontext c = nullptr;
+    return fn(&c) == CUDA_SUCCESS ? c : nullptr;
+}
+
+// Device address of the scratch on the current device.  Looked up once per device (and
+// context) with that device current: in host code the array's name is only a host-side
+// stand-in.
 int scratch_on_current_device(int **out)
 {
     int dev = -1;
@@ -44,13 +68,15 @@ int scratch_on_current_device(int **out)
         return MOE_ENODEV;
     }
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_dev[dev]) {
+    const CUcontext ctx = current_context();
+    if (!g_scratch_dev[dev] || !ctx || ctx != g_scratch_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) {
             cudaGetLastError();
             return MOE_ECUDA;
         }
         g_scratch_dev[dev] = static_cast<int *>(p);
+        g_scratch_ctx[dev] = current_context();   // the lookup made the device's context current
     }
     *out = g_scratch_dev[dev];
     return MOE_OK;

@@ -1,6 +1,7 @@
 // router.cu -- routing logits, softmax and top-2 ("Grok-1 Admin & Architecture Guide",
-// section 3, "Mixture of Experts (MoELayer + Router)", steps 1-2), and the pre-MoE
-// RMSNorm of the residual block ("Transformer stack and language model head").
+// section 3, "Mixture of Experts (MoELayer + Router)", steps 1-2), with the pre-MoE
+// RMSNorm of the residual block ("Transformer stack and language model head") folded in:
+// the routed row is then the normalised one, which the kernel also stores for the gather.
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "route_common.cuh"
@@ -18,7 +19,11 @@ __global__ void __launch_bounds__(kRouteTokenThreads) router_small_kernel(RouteA
 
 // Many tokens: each warp takes 4 tokens, so every router-weight load feeds 4 tokens and
 // the 8 warps of a block share those loads through L1; lane partial sums are reduced
-// with a butterfly (fixed order).
+// with a butterfly (fixed order; every lane ends with the same sum).
+// With a.g_pre set (the residual block), the routed rows are u = bf16(x * rsqrt(mean(x^2) +
+// eps) * g_pre): a first pass takes each token's sum of squares (lane partials over the
+// lane's chunks in order, then the butterfly), the second forms each 8-element chunk of u in
+// fp32, rounds it to bf16, stores it to a.u (for the gather) and routes on it.
 __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouteArgs a)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -31,12 +36,58 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouteArgs a)
 #pragma unroll
         for (int e = 0; e < kExperts; ++e) acc[j][e] = 0.f;
     const int chunks = a.d >> 3;
+    float rn[kTokensPerWarp];   // RMSNorm factor of each token (residual block only)
+    if (a.g_pre) {
+        float ss[kTokensPerWarp];
+#pragma unroll
+        for (int j = 0; j < kTokensPerWarp; ++j) ss[j] = 0.f;
+        for (int c = lane; c < chunks; c += 32) {
+#pragma unroll
+            for (int j = 0; j < kTokensPerWarp; ++j) {
+                const int t = min(t0 + j, a.T - 1);
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * a.d) + c);
+                const uint32_t hv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float lo = __uint_as_float(hv[q] << 16), hi = __uint_as_float(hv[q] & 0xffff0000u);
+                    ss[j] = fmaf(lo, lo, ss[j]);
+                    ss[j] = fmaf(hi, hi, ss[j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kTokensPerWarp; ++j) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], o);
+            rn[j] = rsqrtf(ss[j] / static_cast<float>(a.d) + a.eps);
+        }
+    }
     for (int c = lane; c < chunks; c += 32) {
         uint4 xv[kTokensPerWarp];
 #pragma unroll
         for (int j = 0; j < kTokensPerWarp; ++j) {
             const int t = min(t0 + j, a.T - 1);
             xv[j] = __ldg(reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * a.d) + c);
+        }
+        if (a.g_pre) {
+            const uint4 g = __ldg(reinterpret_cast<const uint4 *>(a.g_pre) + c);
+            const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+            for (int j = 0; j < kTokensPerWarp; ++j) {
+                const uint32_t hv[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+                uint32_t uv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float lo = __uint_as_float(hv[q] << 16) * rn[j] * __uint_as_float(gv[q] << 16);
+                    const float hi =
+                        __uint_as_float(hv[q] & 0xffff0000u) * rn[j] * __uint_as_float(gv[q] & 0xffff0000u);
+                    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+                    uv[q] = *reinterpret_cast<const uint32_t *>(&p);
+                }
+                xv[j] = make_uint4(uv[0], uv[1], uv[2], uv[3]);
+                if (t0 + j < a.T)
+                    reinterpret_cast<uint4 *>(a.u + static_cast<size_t>(t0 + j) * a.d)[c] = xv[j];
+            }
         }
         const uint32_t *wv = reinterpret_cast<const uint32_t *>(xv);
 #pragma unroll
@@ -85,30 +136,6 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_kernel(RouteArgs a)
     }
 }
 
-// u = bf16( h * rsqrt(mean(h^2) + eps) * g ), one block per token, fp32 math.
-__global__ void __launch_bounds__(256) prenorm_kernel(NormArgs a)
-{
-    __shared__ float red[8];
-    const int t = blockIdx.x;
-    const __nv_bfloat16 *hr = a.h + static_cast<size_t>(t) * a.d;
-    float ss = 0.f;
-    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
-        const float v = __bfloat162float(hr[i]);
-        ss = fmaf(v, v, ss);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) tot += red[w];
-    const float r = rsqrtf(tot / static_cast<float>(a.d) + a.eps);
-    __nv_bfloat16 *ur = a.u + static_cast<size_t>(t) * a.d;
-    for (int i = threadIdx.x; i < a.d; i += blockDim.x)
-        ur[i] = __float2bfloat16_rn(__bfloat162float(hr[i]) * r * __bfloat162float(a.g[i]));
-}
-
 }  // namespace
 
 cudaError_t launch_router(const RouteArgs &a, cudaStream_t s)
@@ -123,11 +150,5 @@ cudaError_t launch_router(const RouteArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-cudaError_t launch_prenorm(const NormArgs &a, cudaStream_t s)
-{
-    if (a.T <= 0) return cudaSuccess;
-    prenorm_kernel<<<a.T, 256, 0, s>>>(a);
-    return cudaGetLastError();
-}
 
 }  // namespace moe

@@ -133,3 +133,14 @@ def test_forward_without_gpu_reports_no_device(m):
     finally:
         m.moe_destroy(h)
 
+
+
+def test_block_input_needs_a_block_forward(m):
+    """moe_get_block_input before any forward (here: a handle that never ran) is refused on the host."""
+    rc, h = m.moe_create(256, 512, 8, 2)
+    assert rc == m.MOE_OK
+    try:
+        assert m.moe_get_block_input(h, 1 << 20, 0) == m.MOE_EINVAL
+        assert m.moe_get_block_input(None, 1 << 20, 0) == m.MOE_EINVAL
+    finally:
+        m.moe_destroy(h)

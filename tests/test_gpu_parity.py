@@ -155,37 +155,27 @@ def test_small_batch_routing_is_one_launch(m, tiny_inputs, tiny_handle):
         assert times[k][1] == 0
 
 
-@pytest.mark.parametrize("T", [8, 64])
+@pytest.mark.parametrize("T", [8, 64, 300])
 def test_tiny_residual_block(m, tiny_inputs, tiny_handle, T):
-    """moe_block_forward on the tiny layer with non-unit RMSNorm gains: T=8 takes the
-    pre-norm inside the small-batch routing launch, T=64 the separate pre-norm kernel."""
+    """moe_block_forward on the tiny layer with non-unit RMSNorm gains, checked on the GPU's own
+    MoE input (parity.check_block).  T=8 normalises inside the small-batch routing launch,
+    T=64 inside the one-block-per-token router, T=300 inside the four-tokens-per-warp router:
+    no separate pre-norm launch in any of them."""
     h, layer, _ = tiny_handle
     layer_cpu = parity.to_cpu(tiny_inputs.layers[0])
     g = torch.Generator().manual_seed(11)
     gam = {k: (0.5 + torch.rand(256, generator=g)).to(torch.bfloat16) for k in ("pre", "post")}
     h_in = tiny_inputs.x[:T].clone()
-    chain = oracle.block_chain([layer_cpu], [gam], h_in, eps=1e-5)[0]
     h_dev = h_in.cuda().contiguous()
     m.check(m.moe_set_router_bias(h, None))
+    m.check(m.moe_set_padding_mask(h, None))
+    m.check(m.moe_set_profiling(h, True))
+    m.moe_get_kernel_times(h)
     m.check(m.moe_block_forward(h, T, h_dev, gam["pre"].cuda(), gam["post"].cuda(), 1e-5, *m.layer_args(layer)))
-    idx = torch.empty((T, 2), dtype=torch.int32, device="cuda")
-    m.check(m.moe_get_routing(h, idx))
-    m.check(m.moe_sync_status(h))
-    gidx = idx.cpu().numpy()
-    diff = (gidx != chain["idx"]).any(axis=1)
-    ref_out = chain["h_out"]
-    if diff.any():
-        # the bf16 routed row can round differently after an fp32 vs fp64 RMSNorm; such a
-        # token must be a close call in the oracle, and is compared with the GPU's experts
-        srt = -np.sort(-chain["probs"], axis=1)
-        gap = np.minimum(srt[:, 0] - srt[:, 1], srt[:, 1] - srt[:, 2])
-        assert (gap[diff] < 1e-4).all(), f"routing differs on {np.nonzero(diff)[0]}"
-        forced = [gidx[t] if diff[t] else chain["idx"][t] for t in range(T)]
-        ref_out = oracle.block_chain([layer_cpu], [gam], h_in, eps=1e-5, forced=[np.array(forced)])[0]["h_out"]
-    got = h_dev.cpu().to(torch.float64).numpy()
-    dg, dr = got - chain["h_in"], ref_out - chain["h_in"]
-    err = np.abs(dg - dr).max()
-    assert err <= parity.OUT_RTOL * np.abs(dr).max() + 2 * np.abs(ref_out).max() * 2.0 ** -8, err
+    rc, times = m.moe_get_kernel_times(h)
+    m.check(m.moe_set_profiling(h, False))
+    assert rc == 0 and times["prenorm"][1] == 0
+    parity.check_block(h, T, h_in, h_dev, layer_cpu, gam["pre"], gam["post"], 1e-5)
 
 
 def _padding_mask(T, seed):
@@ -340,6 +330,20 @@ def test_decode_T8_all_tokens(m, grok_handle, grok_layer):
     parity.check_output(run, layer_cpu, x_cpu, range(8), near)
 
 
+def test_decode_T8_rerun_bit_identical(m, grok_handle):
+    """Decode T=8: the packed layout cuts the up-projection's last wave of tiles into K pieces
+    (1792 tiles on 148 CTAs) whose partial sums are added in piece order, and the
+    down-projection splits K 8 ways; two runs on the same inputs give the same bits."""
+    h, layer, _ = grok_handle
+    g = moe_synth.generator(31, "cuda")
+    x = moe_synth.draw_tokens(8, 6144, g, "cuda")
+    m.check(m.moe_set_router_bias(h, None))
+    a = parity.Run(h, x, layer)
+    b = parity.Run(h, x, layer)
+    assert torch.equal(a.out_h, b.out_h)
+    assert np.array_equal(a.perm_h, b.perm_h) and np.array_equal(a.gate_h, b.gate_h)
+
+
 @pytest.mark.parametrize("name,T", [("prefill", 8192), ("skewed", 4096)])
 def test_large_T_sampled(m, grok_handle, grok_layer, name, T):
     grok_handle, layer, _ = grok_handle
@@ -379,11 +383,14 @@ def test_wide_tiles_odd_segments_and_pieces(m, grok_handle, grok_layer):
     near = parity.check_routing(run, ref, 8)
     toks = parity.sample_tokens(run, T, 48)
     parity.check_output(run, layer_cpu, x_cpu, toks, near, bias_cpu=bias)
+    again = parity.Run(h, x, layer, bias.cuda())     # pieces summed in a fixed order: same bits
+    assert torch.equal(again.out_h, run.out_h)
 
 
 def test_stacked_blocks_per_block(m, grok_handle):
     """Four residual blocks, T=32: each block on the GPU is fed the oracle's residual
-    stream (bf16) so that every block is compared on identical inputs."""
+    stream (bf16) so that every block is compared on identical inputs, and is checked on
+    its own MoE input (parity.check_block)."""
     grok_handle, _, layout = grok_handle
     w = moe_synth.WORKLOADS["stacked"]
     inp = moe_synth.make_inputs("stacked", device="cuda")
@@ -393,33 +400,12 @@ def test_stacked_blocks_per_block(m, grok_handle):
     layers_cpu = [parity.to_cpu(l) for l in inp.layers]
     gam_cpu = [{k: v.cpu() for k, v in g.items()} for g in inp.gammas]
     chain = oracle.block_chain(layers_cpu, gam_cpu, inp.x.cpu(), eps=w.eps)
+    m.check(m.moe_set_router_bias(grok_handle, None))
+    m.check(m.moe_set_padding_mask(grok_handle, None))
     for b in range(w.blocks):
         h_in = torch.from_numpy(oracle.f64_to_bf16_bits(chain[b]["h_in"]).view(np.int16)).view(torch.bfloat16)
         h_dev = h_in.cuda().contiguous()
-        m.check(m.moe_set_router_bias(grok_handle, None))
         m.check(m.moe_block_forward(grok_handle, w.T, h_dev, inp.gammas[b]["pre"], inp.gammas[b]["post"], w.eps,
                                     *m.layer_args(layers_dev[b])))
-        idx = torch.empty((w.T, 2), dtype=torch.int32, device="cuda")
-        m.check(m.moe_get_routing(grok_handle, idx))
-        m.check(m.moe_sync_status(grok_handle))
-        gidx = idx.cpu().numpy()
-        # routing: bit-exact outside near ties of the oracle's probabilities
-        near = oracle.near_ties(chain[b]["probs"], parity.NEAR_TIE)
-        diff = (gidx != chain[b]["idx"]).any(axis=1)
-        ref_out = chain[b]["h_out"]
-        if (diff & ~near).any():
-            # the bf16 MoE input of a token can round differently in fp32 vs fp64
-            # RMSNorm; such a token must then be a close call in the oracle too
-            s = -np.sort(-chain[b]["probs"], axis=1)
-            gap = np.minimum(s[:, 0] - s[:, 1], s[:, 1] - s[:, 2])
-            assert (gap[diff] < 1e-4).all(), f"block {b}: routing differs on {np.nonzero(diff)[0]}"
-        if diff.any():
-            forced = [gidx[t] if diff[t] else chain[b]["idx"][t] for t in range(w.T)]
-            redo = oracle.block_chain([layers_cpu[b]], [gam_cpu[b]], h_in, eps=w.eps, forced=[np.array(forced)])
-            ref_out = redo[0]["h_out"]
-        got = h_dev.cpu().to(torch.float64).numpy()
-        # compare the block's contribution h_out - h_in (the residual itself is exact input)
-        dg, dr = got - chain[b]["h_in"], ref_out - chain[b]["h_in"]
-        err = np.abs(dg - dr).max()
-        assert err <= parity.OUT_RTOL * np.abs(dr).max() + 2 * np.abs(ref_out).max() * 2.0 ** -8, \
-            f"block {b}: {err}"
+        parity.check_block(grok_handle, w.T, h_in, h_dev, layers_cpu[b], gam_cpu[b]["pre"], gam_cpu[b]["post"],
+                           w.eps)
