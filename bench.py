@@ -68,6 +68,9 @@ def parse(argv=None):
                    help="weight scale format: 0 per output channel, 128 per block of 128 inputs (packed layout)")
     p.add_argument("--layout", choices=("packed", "in_out"), default="packed",
                    help="weight layout: packed = tiles written once at load (TMEM path); in_out = as drawn")
+    p.add_argument("--parallel", choices=("replicas", "ep"), default="replicas",
+                   help="several GPUs: independent replicas (default), or experts spread over the ranks "
+                        "(each rank E/N experts and its own tokens; all-to-all exchanges over NCCL)")
     return p.parse_args(argv)
 
 
@@ -91,7 +94,7 @@ def dist_setup(n_gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    if world > 1 or "MASTER_ADDR" in os.environ:   # under torchrun (a one-rank group included)
         import datetime
         import torch.distributed as dist
         backend = os.environ.get("MOE_BENCH_BACKEND", "nccl")
@@ -129,8 +132,8 @@ def job_value(tokens_per_rank: int, world: int, ms_per_rank: float, device=None)
 
 
 def dist_teardown(world: int):
-    if world > 1:
-        import torch.distributed as dist
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
         dist.destroy_process_group()
 
 
@@ -466,10 +469,75 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
     return rec, launches_per_step
 
 
+def bench_ep(args, world, rank, dev):
+    """Expert parallelism: rank r holds experts [r*E/N, (r+1)*E/N) of the one model and its own
+    T tokens; a step is the whole layer on every rank, exchanges included (all-to-all over the
+    default process group).  Needs torch.distributed (torchrun), any N that divides E."""
+    import torch
+    import torch.distributed as dist
+    import moe_synth
+    import mixture_experts_softmax_b200 as moe
+    from mixture_experts_softmax_b200 import ep
+
+    name = args.workload or "prefill"
+    w = moe_synth.WORKLOADS[name]
+    if w.blocks or w.bias is not None:
+        raise SystemExit("--parallel ep runs the plain layer workloads (prefill, decode)")
+    if not dist.is_initialized():
+        raise SystemExit("--parallel ep needs torchrun (a process group), also for one GPU")
+    ks, ws = default_steps(name)
+    K = args.steps if args.steps is not None else ks
+    W = max(3, args.warmup if args.warmup is not None else ws)
+    full = moe_synth.make_inputs(w, device=dev).layers[0]          # the same model on every rank
+    first, last = ep.expert_range(w.E, world, rank)
+    rk = ep.EPRank(w.d, w.F, world, rank, ep.slice_experts(full, first, last), E=w.E, packed=args.layout == "packed")
+    del full
+    torch.cuda.empty_cache()
+    x = moe_synth.draw_tokens(w.T, w.d, moe_synth.generator(w.seed + 1000 + rank, dev), dev)
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(W):
+        rk.forward(x, out)
+    moe.check(moe.moe_sync_status(rk.layer.h, stream))
+    R = int(max_over_ranks(args.repeats or 3, world, dev))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    region_ms = []
+    for r in range(R):
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        if clocks and r == 0:
+            clocks.mark("t0")
+        e0.record(stream)
+        for _ in range(K):
+            rk.forward(x, out)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        region_ms.append(e0.elapsed_time(e1))
+    if clocks:
+        clocks.mark("t1")
+    barrier(world, dev)
+    clk = clocks.stop() if clocks else None
+    moe.check(moe.moe_sync_status(rk.layer.h, stream))
+    value, ms_max = job_value(w.T, world, statistics.median(region_ms) / K, dev)
+    rk.close()
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+            "repeats": R, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": DATA, "clocks": clk,
+            "config": {"workload": name, "T_per_gpu": w.T, "d_model": w.d, "ffn": w.F, "experts": w.E,
+                       "top_k": w.k, "parallelism": f"expert parallel x{world} ({w.E // world} experts per rank)",
+                       "exchange": "torch.distributed all_to_all_single (counts, bf16 rows, fp32 results)",
+                       "weights": "int8 + bf16 per-output-channel scales, layout " + args.layout}}
+
+
 def run_native(args, world, rank, local):
     import torch
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.parallel == "ep":
+        return bench_ep(args, world, rank, dev)
     head = args.workload or "prefill"
     with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
     rec, lps = bench_workload(head, args, world, rank, dev, args.layout, args.cpu_seconds, with_cpu)

@@ -263,6 +263,70 @@ MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int
  */
 MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits);
 
+/*
+ * Expert parallelism: the experts spread over W ranks, as the pages' own layout spreads
+ * them over the `model` mesh axis ("Grok-1 Admin & Architecture Guide", section 6
+ * "Sharding & Parallelism Deep Dive", the MoE matmuls under shard_map).  Rank r of W
+ * holds E_local = E / W consecutive experts, [r * E_local, (r + 1) * E_local), and its
+ * own tokens.  One layer is three device steps on each rank, with two exchanges between
+ * ranks that the caller makes (all-to-all; the Python package does it with
+ * torch.distributed over NCCL):
+ *
+ *   moe_ep_dispatch   route the rank's T tokens; routed rows grouped by expert (hence by
+ *                     destination rank) into send_rows, per-expert row counts;
+ *   exchange          counts, then rows: rank j receives, from every source s in rank
+ *                     order, s's rows for j's experts (in s's order);
+ *   moe_ep_experts    the rank's experts on the rows it received -> y rows, same order;
+ *   exchange          y rows back to their sources (the reverse of the row exchange);
+ *   moe_ep_combine    out[t] = gate0 * y(t, slot 0) + gate1 * y(t, slot 1).
+ *
+ * The result is the layer of moe_forward on the rank's tokens.  The handle keeps the
+ * dispatch's routing until moe_ep_combine; a moe_forward / moe_block_forward on the same
+ * handle in between discards it.
+ */
+
+/*
+ * Step 1: routing ("Mixture of Experts (MoELayer + Router)", steps 1-2, with the handle's
+ * router bias and padding mask) and grouping of this rank's T tokens.
+ *   x            bf16 [T, d]   this rank's tokens
+ *   router_w     fp32 [d, E]   the full router (every rank routes over all E experts)
+ *   send_rows    bf16 [2T, d]  out: row i = x[perm[i] / 2] for the n = sum(send_counts)
+ *                              routed rows, grouped by expert, ascending token order within one
+ *   send_counts  int32 [E]     out (device): routed rows per expert
+ * moe_get_routing then reports this routing (perm = the order of send_rows).  Returns
+ * MOE_EINVAL on a bad argument, MOE_ECUDA if a launch failed.  T == 0 only sets the
+ * counts to 0 (x and send_rows may then be NULL).
+ */
+MOE_API int moe_ep_dispatch(moe_handle h, int T, const void *x, const float *router_w, void *send_rows,
+                            int32_t *send_counts, void *stream);
+
+/*
+ * Step 3: the rank's E_local experts (step 3 of the MoE section: linear_1(gelu(linear(x)) *
+ * linear_v(x)), 8-bit weights) on the rows it received.
+ *   recv_counts  int32 [n_src, E_local]  HOST array: rows received from source rank s for
+ *                                       local expert k (what the count exchange delivered)
+ *   recv_rows    bf16 [R, d]   the received rows, R = sum(recv_counts): source after source,
+ *                              each source's rows grouped by local expert
+ *   weights      the E_local experts' w_lin, s_lin, w_v, s_v, w_1, s_1 in the handle's
+ *                weight layout and scale format ([E_local, ...] in place of [E, ...])
+ *   y_rows       fp32 [R, d]   out: row i = s_1 * (H_i . W_1) of received row i's expert
+ *                              (not gate-weighted: the source applies the gates)
+ * Returns MOE_EUNSUPPORTED if n_src * E_local > 64, MOE_EINVAL on a bad argument or
+ * R > 2 * MOE_MAX_TOKENS.  R == 0 is a no-op.
+ */
+MOE_API int moe_ep_experts(moe_handle h, int n_src, int E_local, const int32_t *recv_counts, const void *recv_rows,
+                           const int8_t *w_lin, const void *s_lin, const int8_t *w_v, const void *s_v,
+                           const int8_t *w_1, const void *s_1, float *y_rows, void *stream);
+
+/*
+ * Step 5: the gate-weighted combine of step 4 of the MoE section, in slot order.
+ *   y_back  fp32 [n, d]   the y rows of this rank's sent rows, back in send_rows order
+ *   out     bf16 [T, d]   out[t] = bf16(gate[t,0] * y(t,0) + gate[t,1] * y(t,1)); 0 for a
+ *                         padding token
+ * T must be the T of the handle's last moe_ep_dispatch (else MOE_EINVAL).
+ */
+MOE_API int moe_ep_combine(moe_handle h, int T, const float *y_back, void *out, void *stream);
+
 /* Largest token count moe_route_noalloc accepts (its static scratch is sized for it). */
 #define MOE_NOALLOC_MAX_TOKENS 65536
 

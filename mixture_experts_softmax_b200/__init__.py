@@ -40,6 +40,7 @@ EXPORTS = (
     "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing", "moe_get_block_input",
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
     "moe_set_weight_layout", "moe_pack_weight", "moe_route_noalloc",
+    "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
 )
 
 
@@ -77,6 +78,9 @@ def _load() -> ctypes.CDLL:
         "moe_set_weight_layout": (I, [P, I]),
         "moe_pack_weight": (I, [P, P, P, I, P]),
         "moe_route_noalloc": (I, [I, I, P, P, P, P, P, P, P, P]),
+        "moe_ep_dispatch": (I, [P, I, P, P, P, P, P]),
+        "moe_ep_experts": (I, [P, I, I, P, P, P, P, P, P, P, P, P, P]),
+        "moe_ep_combine": (I, [P, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -221,6 +225,27 @@ def pack_layer(h, layer: dict, stream=None) -> dict:
 def moe_route_noalloc(T, d, x, router_w, bias, idx, gate, offsets, perm, stream=None) -> int:
     return _lib.moe_route_noalloc(int(T), int(d), _ptr(x), _ptr(router_w), _ptr(bias), _ptr(idx), _ptr(gate),
                                   _ptr(offsets), _ptr(perm), _stream(stream))
+
+
+def moe_ep_dispatch(h, T, x, router_w, send_rows, send_counts, stream=None) -> int:
+    return _lib.moe_ep_dispatch(h, int(T), _ptr(x), _ptr(router_w), _ptr(send_rows), _ptr(send_counts),
+                                _stream(stream))
+
+
+def moe_ep_experts(h, n_src, E_local, recv_counts, recv_rows, w_lin, s_lin, w_v, s_v, w_1, s_1, y_rows,
+                   stream=None) -> int:
+    """recv_counts: HOST int32 [n_src, E_local] (a CPU tensor or a sequence of ints)."""
+    import torch
+    rc = torch.as_tensor(recv_counts, dtype=torch.int32).contiguous()
+    if rc.device.type != "cpu":
+        raise ValueError("recv_counts must be on the host")
+    return _lib.moe_ep_experts(h, int(n_src), int(E_local), rc.data_ptr(), _ptr(recv_rows), _ptr(w_lin),
+                               _ptr(s_lin), _ptr(w_v), _ptr(s_v), _ptr(w_1), _ptr(s_1), _ptr(y_rows),
+                               _stream(stream))
+
+
+def moe_ep_combine(h, T, y_back, out, stream=None) -> int:
+    return _lib.moe_ep_combine(h, int(T), _ptr(y_back), _ptr(out), _stream(stream))
 
 
 def moe_plan(h, T: int):

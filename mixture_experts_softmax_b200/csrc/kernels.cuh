@@ -97,6 +97,36 @@ struct CombineArgs {
 };
 
 
+// expert-parallel steps (ep.cu)
+constexpr int kEpMaxRuns = 64;   // n_src * E_local: (source rank, local expert) pairs
+struct EpLayoutArgs {
+    int n_src, E_local, bn, R;  // R = the sum of recv_counts
+    int recv_counts[kEpMaxRuns]; // [n_src, E_local] rows received from each source for each local expert
+    int *counts;                // [E_local]
+    int *offsets;               // [E_local + 1] unpadded grouped offsets
+    int *poff;                  // [E_local + 1] offsets with each expert's segment padded to bn rows
+    int *rperm;                 // [rows] padded grouped row -> received row, -1 for padding
+    int *slot;                  // [R] received row -> padded grouped row
+    float *ones;                // [R] set to 1: the GEMMs' gate (the source applies the real gates)
+};
+
+struct EpCombineArgs {
+    int T, d;
+    const int *idx;             // [T, 2] experts (-1: padding token)
+    const float *gate;          // [T, 2]
+    const int *slot_of_route;   // [2T] route -> its row in the sent (and returned) order
+    const float *y;             // [rows sent, d] expert outputs returned by their ranks
+    __nv_bfloat16 *out;         // [T, d]
+};
+
+cudaError_t launch_ep_layout(const EpLayoutArgs &a, cudaStream_t s);
+// xp[slot[i]] = rows[i], i < R
+cudaError_t launch_ep_gather(int R, int d, const __nv_bfloat16 *rows, const int *slot, __nv_bfloat16 *xp,
+                             cudaStream_t s);
+// y[i] = sum_s part[s * plane + i * d ...], s ascending
+cudaError_t launch_ep_split_sum(int R, int d, int splits, size_t plane, const float *part, float *y, cudaStream_t s);
+cudaError_t launch_ep_combine(const EpCombineArgs &a, cudaStream_t s);
+
 cudaError_t launch_router(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 // Xp[slot_of_route[r]] = x[r / 2] for the 2T routes

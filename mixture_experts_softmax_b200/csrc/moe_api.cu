@@ -25,6 +25,7 @@ struct WeightMap {
     const void *ptr = nullptr;
     int kind = -1;     // 0: linear / linear_v   1: linear_1
     int layout = -1;   // MOE_LAYOUT_IN_OUT or MOE_LAYOUT_PACKED
+    int experts = 0;   // experts in the tensor
     CUtensorMap map;
 };
 
@@ -58,6 +59,8 @@ struct moe_ctx {
     int map_gen = 0;        // bumps when b_xp / b_h move
     int last_T = -1;
     int last_block_T = -1;  // T of the last forward if it was moe_block_forward (u is staged), else -1
+    int ep_T = -1;          // T of the last moe_ep_dispatch (its routing waits for moe_ep_combine), else -1
+    DevBuf b_ep;            // expert-parallel layout of received rows: counts, offsets, poff, rperm, slot, ones
 
     // TMA descriptors
     std::vector<WeightMap> wmaps;
@@ -101,6 +104,19 @@ int bn_slot(int bn) { return bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3; }
 int kstage_of(const moe_ctx *h, bool up, int bn)
 {
     return h->layout == MOE_LAYOUT_PACKED ? gemm_ts_kstage(up, bn) : kBK;
+}
+
+// K-splits of the down-projection: double while the tiles of `experts` experts with about
+// `per_expert` rows each fill fewer than 16 waves and the stages still divide evenly
+int splits_for(const moe_ctx *h, int experts, int per_expert, int bn)
+{
+    const long nt = per_expert <= bn ? 1 : (per_expert + bn - 1) / bn;
+    const long tiles = static_cast<long>(experts) * (h->d / kBM) * nt;
+    const int ksteps = h->F / kstage_of(h, false, bn);
+    const int sms = h->num_sms > 0 ? h->num_sms : 148;
+    int s = 1;
+    while (s < kMaxSplits && tiles * s < 16L * sms && ksteps % (2 * s) == 0) s *= 2;
+    return s;
 }
 
 int plan_splits(const moe_ctx *h, int T, int bn)
@@ -198,22 +214,27 @@ int ensure_device(moe_ctx *h)
     return MOE_OK;
 }
 
+// grouped-row buffers (rperm, Xp, H) for at least `rows` rows
+int ensure_rows(moe_ctx *h, int rows)
+{
+    int rc;
+    if (rows > h->rows_cap) {
+        if ((rc = ensure(h, h->b_rperm, static_cast<size_t>(rows) * 4)) != MOE_OK) return rc;
+        if ((rc = ensure(h, h->b_xp, static_cast<size_t>(rows) * h->d * 2)) != MOE_OK) return rc;
+        if ((rc = ensure(h, h->b_h, static_cast<size_t>(rows) * h->F * 2)) != MOE_OK) return rc;
+        h->rows_cap = rows;
+        // the descriptors cover rows_cap rows: rebuild them all
+        h->map_gen++;
+    }
+    return MOE_OK;
+}
+
 int ensure_workspace(moe_ctx *h, int T, int bn, int splits)
 {
     int rc;
     const RouteLayout L = route_layout(T, h->E);
     if ((rc = ensure(h, h->b_route, L.words * 4)) != MOE_OK) return rc;
-    const int rows = rows_for(h, T, bn);
-    bool moved = false;
-    if (rows > h->rows_cap) {
-        if ((rc = ensure(h, h->b_rperm, static_cast<size_t>(rows) * 4)) != MOE_OK) return rc;
-        if ((rc = ensure(h, h->b_xp, static_cast<size_t>(rows) * h->d * 2, &moved)) != MOE_OK) return rc;
-        if ((rc = ensure(h, h->b_h, static_cast<size_t>(rows) * h->F * 2, &moved)) != MOE_OK) return rc;
-        h->rows_cap = rows;
-        // the descriptors cover rows_cap rows: rebuild them all
-        h->map_gen++;
-    }
-    (void)moved;
+    if ((rc = ensure_rows(h, rows_for(h, T, bn))) != MOE_OK) return rc;
     if ((rc = ensure(h, h->b_slots, static_cast<size_t>(splits) * T * 2 * h->d * 4)) != MOE_OK) return rc;
     if ((rc = ensure(h, h->b_stage, static_cast<size_t>(T) * h->d * 2 * 2)) != MOE_OK) return rc;
     // last-wave partial sums of the TMEM GEMMs: one 128-row tile of up to 256 fp32 columns per SM
@@ -257,10 +278,12 @@ int encode_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *ptr
 // [E, out, in] (packed) layout: rows = E*out, box = 128 feature-rows x 128 k.
 // The tensor map of a weight, from the handle's cache (encoded on first use).  The map is
 // copied out: a pointer into the cache would dangle once a later insertion moves it.
-int weight_map(moe_ctx *h, const void *ptr, int kind, CUtensorMap *out)
+// E_w: experts the weight tensor holds (the handle's E, or a rank's local experts)
+int weight_map(moe_ctx *h, const void *ptr, int kind, CUtensorMap *out, int E_w = 0)
 {
+    if (E_w <= 0) E_w = h->E;
     for (auto &w : h->wmaps)
-        if (w.ptr == ptr && w.kind == kind && w.layout == h->layout) {
+        if (w.ptr == ptr && w.kind == kind && w.layout == h->layout && w.experts == E_w) {
             *out = w.map;
             return MOE_OK;
         }
@@ -268,13 +291,14 @@ int weight_map(moe_ctx *h, const void *ptr, int kind, CUtensorMap *out)
     w.ptr = ptr;
     w.kind = kind;
     w.layout = h->layout;
+    w.experts = E_w;
     const uint64_t in = kind == 0 ? h->d : h->F, outf = kind == 0 ? h->F : h->d;
     int rc;
     if (h->layout == MOE_LAYOUT_PACKED)
-        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, in, static_cast<uint64_t>(h->E) * outf,
+        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, in, static_cast<uint64_t>(E_w) * outf,
                        128, kBM);
     else
-        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, outf, static_cast<uint64_t>(h->E) * in,
+        rc = encode_2d(&w.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, outf, static_cast<uint64_t>(E_w) * in,
                        kBM, kBK);
     if (rc != MOE_OK) return rc;
     if (h->wmaps.size() >= 64) h->wmaps.erase(h->wmaps.begin());
@@ -476,6 +500,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
         return MOE_ECUDA;
 
     h->last_block_T = g_pre ? T : -1;
+    h->ep_T = -1;   // the route buffer now holds this forward's routing
     CombineArgs ca{T, h->d, splits, static_cast<const float *>(h->b_slots.ptr), idx, static_cast<__nv_bfloat16 *>(out),
                    static_cast<__nv_bfloat16 *>(h_io), static_cast<const __nv_bfloat16 *>(g_post), eps};
     if (timed(h, K_COMBINE, s, [&] { return launch_combine(ca, s); }) != cudaSuccess) return MOE_ECUDA;
@@ -495,6 +520,162 @@ int begin_call(moe_ctx *h, int T, cudaStream_t s)
     if ((rc = ensure_workspace(h, T, bn, plan_splits(h, T, bn))) != MOE_OK) return rc;
     h->last_stream = s;
     h->used = true;
+    return MOE_OK;
+}
+
+// ---- expert parallelism (device steps; the exchange between ranks is the caller's) ----------
+
+// the expert-parallel layout arrays in b_ep, in 4-byte words
+struct EpLayout {
+    size_t counts, offsets, poff, rperm, slot, ones, words;
+};
+
+EpLayout ep_layout(int rows, int R)
+{
+    auto up = [](size_t v) { return (v + 63) / 64 * 64; };
+    EpLayout L;
+    size_t o = 0;
+    L.counts = o; o += 64;
+    L.offsets = o; o += 128;
+    L.poff = o; o += 128;
+    L.rperm = o; o += up(rows);
+    L.slot = o; o += up(R);
+    L.ones = o; o += up(R);
+    L.words = o;
+    return L;
+}
+
+// routing + grouping by expert (no padding: grouped row i is route perm[i]) + the routed rows
+// gathered into send_rows in that order
+int run_ep_dispatch(moe_ctx *h, int T, const void *x, const float *router_w, void *send_rows, int32_t *send_counts,
+                    cudaStream_t s)
+{
+    const RouteLayout L = route_layout(T, h->E);
+    int *rw = static_cast<int *>(h->b_route.ptr);
+    int *idx = rw + L.idx;
+    float *gate = reinterpret_cast<float *>(rw + L.gate);
+    RouteArgs ra{T, h->d, static_cast<const __nv_bfloat16 *>(x), router_w, h->bias, idx, gate};
+    ra.mask = h->mask;
+    DispatchArgs da{T, h->E, 1, idx, rw + L.counts, rw + L.offsets, rw + L.poff, rw + L.perm,
+                    static_cast<int *>(h->b_rperm.ptr), rw + L.slot};
+    GatherArgs ga{h->d, static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(send_rows)};
+    if (T <= route_small_max_tokens()) {
+        unsigned int *ticket = reinterpret_cast<unsigned int *>(h->err + kCtlRouteTicket);
+        float *part = static_cast<float *>(h->b_slots.ptr);
+        const int S = route_small_slices(T, h->d, h->num_sms);
+        if (timed(h, K_ROUTE_SMALL, s, [&] { return launch_route_small(ra, da, ga, part, S, ticket, s); }) !=
+            cudaSuccess)
+            return MOE_ECUDA;
+    } else {
+        if (timed(h, K_ROUTER, s, [&] { return launch_router(ra, s); }) != cudaSuccess) return MOE_ECUDA;
+        if (timed(h, K_DISPATCH, s, [&] { return launch_dispatch(da, s); }) != cudaSuccess) return MOE_ECUDA;
+        if (timed(h, K_GATHER, s, [&] { return launch_gather(ga, T, rw + L.slot, s); }) != cudaSuccess)
+            return MOE_ECUDA;
+    }
+    if (cudaMemcpyAsync(send_counts, rw + L.counts, static_cast<size_t>(h->E) * 4, cudaMemcpyDeviceToDevice, s) !=
+        cudaSuccess)
+        return MOE_ECUDA;
+    h->last_T = T;
+    h->last_block_T = -1;
+    h->ep_T = T;
+    return MOE_OK;
+}
+
+int run_ep_experts(moe_ctx *h, int n_src, int E_local, const int32_t *counts, int R, int max_rows,
+                   const void *recv_rows, const int8_t *w_lin, const void *s_lin, const int8_t *w_v, const void *s_v,
+                   const int8_t *w_1, const void *s_1, float *y_rows, cudaStream_t s)
+{
+    int rc;
+    const int bn = max_rows <= 16 ? 16 : max_rows <= 32 ? 32 : max_rows <= 64 ? 64 : 128;
+    const int splits = splits_for(h, E_local, max_rows, bn);
+    const int Tp = (R + 1) / 2;   // the down-projection's slots [splits, Tp, 2, d] hold rows [splits, 2 Tp, d]
+    const int rows = ((R + E_local * (bn - 1)) + 127) / 128 * 128;
+    if ((rc = ensure_rows(h, rows)) != MOE_OK) return rc;
+    if (splits > 1 && (rc = ensure(h, h->b_slots, static_cast<size_t>(splits) * Tp * 2 * h->d * 4)) != MOE_OK)
+        return rc;
+    if (h->layout == MOE_LAYOUT_PACKED &&
+        (rc = ensure(h, h->b_part, static_cast<size_t>(h->num_sms) * 128 * 256 * 4)) != MOE_OK)
+        return rc;
+    const EpLayout L = ep_layout(h->rows_cap, R);
+    if ((rc = ensure(h, h->b_ep, L.words * 4)) != MOE_OK) return rc;
+
+    const bool ts = h->layout == MOE_LAYOUT_PACKED;
+    if (h->kblock && !ts) return MOE_EUNSUPPORTED;
+    CUtensorMap m_wl, m_wv, m_w1;
+    const CUtensorMap *m_xp, *m_h;
+    if ((rc = weight_map(h, w_lin, 0, &m_wl, E_local)) != MOE_OK) return rc;
+    if ((rc = weight_map(h, w_v, 0, &m_wv, E_local)) != MOE_OK) return rc;
+    if ((rc = weight_map(h, w_1, 1, &m_w1, E_local)) != MOE_OK) return rc;
+    if ((rc = act_maps(h, bn, &m_xp, &m_h)) != MOE_OK) return rc;
+
+    int *ew = static_cast<int *>(h->b_ep.ptr);
+    float *ones = reinterpret_cast<float *>(ew + L.ones);
+    EpLayoutArgs la{};
+    la.n_src = n_src;
+    la.E_local = E_local;
+    la.bn = bn;
+    la.R = R;
+    for (int i = 0; i < n_src * E_local; ++i) la.recv_counts[i] = counts[i];
+    la.counts = ew + L.counts;
+    la.offsets = ew + L.offsets;
+    la.poff = ew + L.poff;
+    la.rperm = ew + L.rperm;
+    la.slot = ew + L.slot;
+    la.ones = ones;
+    if (timed(h, K_DISPATCH, s, [&] { return launch_ep_layout(la, s); }) != cudaSuccess) return MOE_ECUDA;
+    if (timed(h, K_GATHER, s, [&] {
+            return launch_ep_gather(R, h->d, static_cast<const __nv_bfloat16 *>(recv_rows), la.slot,
+                                    static_cast<__nv_bfloat16 *>(h->b_xp.ptr), s);
+        }) != cudaSuccess)
+        return MOE_ECUDA;
+
+    GemmArgs up{};
+    up.T = Tp;
+    up.E = E_local;
+    up.M = h->F;
+    up.K = h->d;
+    up.ksteps = h->d / kstage_of(h, true, bn);
+    up.splits = 1;
+    up.poff = la.poff;
+    up.offsets = la.offsets;
+    up.rperm = la.rperm;
+    up.gate = ones;
+    up.s0 = static_cast<const __nv_bfloat16 *>(s_lin);
+    up.s1 = static_cast<const __nv_bfloat16 *>(s_v);
+    up.h = static_cast<__nv_bfloat16 *>(h->b_h.ptr);
+    up.err = h->err;
+    up.timeout_ns = h->timeout_ns;
+    up.kblock = h->kblock;
+    up.gather = 0;
+    if (ts) {
+        up.part = static_cast<float *>(h->b_part.ptr);
+        up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
+    }
+    if (timed(h, K_UP, s, [&] {
+            return ts ? launch_gemm_up_ts(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s)
+                      : launch_gemm_up(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s);
+        }) != cudaSuccess)
+        return MOE_ECUDA;
+    GemmArgs dn = up;
+    dn.M = h->d;
+    dn.K = h->F;
+    dn.splits = splits;
+    dn.ksteps = h->F / kstage_of(h, false, bn) / splits;
+    dn.s0 = static_cast<const __nv_bfloat16 *>(s_1);
+    dn.s1 = nullptr;
+    dn.h = nullptr;
+    // one split: route id i lands in row i of [Tp, 2, d] = y_rows itself
+    dn.slots = splits == 1 ? y_rows : static_cast<float *>(h->b_slots.ptr);
+    if (timed(h, K_DOWN, s, [&] {
+            return ts ? launch_gemm_down_ts(bn, m_w1, *m_h, dn, h->num_sms, s)
+                      : launch_gemm_down(bn, m_w1, *m_h, dn, h->num_sms, s);
+        }) != cudaSuccess)
+        return MOE_ECUDA;
+    if (splits > 1 && timed(h, K_COMBINE, s, [&] {
+            return launch_ep_split_sum(R, h->d, splits, static_cast<size_t>(Tp) * 2 * h->d,
+                                       static_cast<const float *>(h->b_slots.ptr), y_rows, s);
+        }) != cudaSuccess)
+        return MOE_ECUDA;
     return MOE_OK;
 }
 
@@ -539,7 +720,7 @@ MOE_API int moe_destroy(moe_handle h)
 {
     if (!h) return MOE_OK;
     sync_last(h);
-    for (DevBuf *b : {&h->b_route, &h->b_rperm, &h->b_xp, &h->b_h, &h->b_slots, &h->b_stage})
+    for (DevBuf *b : {&h->b_route, &h->b_rperm, &h->b_xp, &h->b_h, &h->b_slots, &h->b_stage, &h->b_ep})
         if (b->ptr) cudaFree(b->ptr);
     if (h->err) cudaFree(h->err);
     if (h->b_part.ptr) cudaFree(h->b_part.ptr);
@@ -739,6 +920,76 @@ MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n)
     }
     h->pending.clear();
     return rc;
+}
+
+MOE_API int moe_ep_dispatch(moe_handle h, int T, const void *x, const float *router_w, void *send_rows,
+                            int32_t *send_counts, void *stream)
+{
+    if (!h || T < 0 || T > MOE_MAX_TOKENS) return MOE_EINVAL;
+    if (!send_counts || !aligned16(send_counts)) return MOE_EINVAL;
+    if (T == 0) {   // nothing to route: every count is 0
+        h->ep_T = 0;
+        return cudaMemsetAsync(send_counts, 0, static_cast<size_t>(h->E) * 4, static_cast<cudaStream_t>(stream)) ==
+                       cudaSuccess
+                   ? MOE_OK
+                   : MOE_ECUDA;
+    }
+    if (!x || !router_w || !send_rows) return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(send_rows) || !aligned16(send_counts)) return MOE_EINVAL;
+    const size_t xb = static_cast<size_t>(T) * h->d * 2;
+    if (overlaps(x, xb, send_rows, 2 * xb)) return MOE_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int rc = begin_call(h, T, s);
+    if (rc != MOE_OK) return rc;
+    return run_ep_dispatch(h, T, x, router_w, send_rows, send_counts, s);
+}
+
+MOE_API int moe_ep_experts(moe_handle h, int n_src, int E_local, const int32_t *recv_counts, const void *recv_rows,
+                           const int8_t *w_lin, const void *s_lin, const int8_t *w_v, const void *s_v,
+                           const int8_t *w_1, const void *s_1, float *y_rows, void *stream)
+{
+    if (!h || n_src < 1 || E_local < 1 || E_local > h->E || !recv_counts) return MOE_EINVAL;
+    if (static_cast<long>(n_src) * E_local > kEpMaxRuns) return MOE_EUNSUPPORTED;
+    long R = 0, max_rows = 0;
+    for (int k = 0; k < E_local; ++k) {
+        long n = 0;
+        for (int src = 0; src < n_src; ++src) {
+            const int c = recv_counts[src * E_local + k];
+            if (c < 0) return MOE_EINVAL;
+            n += c;
+        }
+        max_rows = n > max_rows ? n : max_rows;
+        R += n;
+    }
+    if (R > 2L * MOE_MAX_TOKENS) return MOE_EINVAL;   // more rows than the workspace plans for
+    if (R == 0) return MOE_OK;
+    if (!recv_rows || !y_rows || !aligned16(recv_rows) || !aligned16(y_rows)) return MOE_EINVAL;
+    const void *ws[] = {w_lin, s_lin, w_v, s_v, w_1, s_1};
+    for (const void *p : ws)
+        if (!p || !aligned16(p)) return MOE_EINVAL;
+    int rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((rc = ensure_device(h)) != MOE_OK) return rc;
+    if (h->used && s != h->last_stream && cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
+    h->last_stream = s;
+    h->used = true;
+    return run_ep_experts(h, n_src, E_local, recv_counts, static_cast<int>(R), static_cast<int>(max_rows), recv_rows,
+                          w_lin, s_lin, w_v, s_v, w_1, s_1, y_rows, s);
+}
+
+MOE_API int moe_ep_combine(moe_handle h, int T, const float *y_back, void *out, void *stream)
+{
+    if (!h || T < 0 || T != h->ep_T) return MOE_EINVAL;
+    if (T == 0) return MOE_OK;
+    if (!y_back || !out || !aligned16(y_back) || !aligned16(out)) return MOE_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (s != h->last_stream && cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
+    h->last_stream = s;
+    const RouteLayout L = route_layout(T, h->E);
+    const int *rw = static_cast<const int *>(h->b_route.ptr);
+    EpCombineArgs ca{T, h->d, rw + L.idx, reinterpret_cast<const float *>(rw + L.gate), rw + L.slot, y_back,
+                     static_cast<__nv_bfloat16 *>(out)};
+    return timed(h, K_COMBINE, s, [&] { return launch_ep_combine(ca, s); }) == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 }  // extern "C"
