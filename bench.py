@@ -68,6 +68,8 @@ def parse(argv=None):
                    help="weight scale format: 0 per output channel, 128 per block of 128 inputs (packed layout)")
     p.add_argument("--layout", choices=("packed", "in_out"), default="packed",
                    help="weight layout: packed = tiles written once at load (TMEM path); in_out = as drawn")
+    p.add_argument("--no-cta-pairs", action="store_true",
+                   help="up-projection of 128-route tiles on one CTA per tile instead of CTA pairs (comparison)")
     p.add_argument("--parallel", choices=("replicas", "ep"), default="replicas",
                    help="several GPUs: independent replicas (default), or experts spread over the ranks "
                         "(each rank E/N experts and its own tokens; all-to-all exchanges over NCCL)")
@@ -221,7 +223,7 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-GEMM_SOURCES = {"packed": ("gemm_ts.cu", "gemm_common.cuh", "ptx.cuh", "kernels.cuh"),
+GEMM_SOURCES = {"packed": ("gemm_ts.cu", "gemm_ts2.cu", "gemm_common.cuh", "ptx.cuh", "kernels.cuh"),
                 "in_out": ("gemm.cu", "gemm_common.cuh", "ptx.cuh", "kernels.cuh")}
 
 
@@ -315,6 +317,7 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
     stream = torch.cuda.current_stream(dev)
 
     h = moe.MoELayer(w.d, w.F, w.E, w.k)
+    moe.check(moe.moe_set_cta_pairs(h.h, not args.no_cta_pairs))
     moe.check(moe.moe_set_router_bias(h.h, inp.bias))
     moe.check(moe.moe_set_scale_block(h.h, args.scale_block))
     if layout == "packed":
@@ -386,6 +389,7 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
                                  ", layout " + layout +
                                  (" (packed once at load, untimed)" if layout == "packed" else " (as drawn)"),
                       "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],
+                      "cta_pairs": not args.no_cta_pairs,
                       "down_splits": moe.moe_plan(h.h, T)[2]},
            "clocks": clk}
 

@@ -249,6 +249,17 @@ MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
 MOE_API int moe_set_weight_layout(moe_handle h, int layout);
 
 /*
+ * Up-projection of large batches (128-route tiles, MOE_LAYOUT_PACKED, ffn a multiple of
+ * 256) on CTA pairs: one tcgen05 MMA of 256 output features spans the two SMs of a
+ * two-CTA cluster, each SM converting its 128 features' weights and holding half of the
+ * 128 routes' activations, which halves the activation traffic through each SM's shared
+ * memory.  on = 1 (the default) uses pairs where the device can run a full wave of them;
+ * on = 0 keeps one CTA per tile.  Both compute the same sums (same order along the
+ * reduction), so the results are the same.  Returns MOE_EINVAL for a NULL handle.
+ */
+MOE_API int moe_set_cta_pairs(moe_handle h, int on);
+
+/*
  * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT to MOE_LAYOUT_PACKED
  * (a per-expert transpose; values copied unchanged), enqueued on `stream`.
  *   which = 0: w is linear or linear_v, [E, d, F] -> w_packed [E, F, d]
@@ -256,6 +267,15 @@ MOE_API int moe_set_weight_layout(moe_handle h, int layout);
  * w and w_packed are device buffers of E*d*F bytes that must not overlap.
  */
 MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream);
+
+/*
+ * moe_pack_weight for a tensor of n_experts experts (1 <= n_experts <= E): [n, d, F] ->
+ * [n, F, d] (which = 0) or [n, F, d] -> [n, d, F] (which = 1).  An expert-parallel rank
+ * packs its own E / W experts with it.  Buffers of n_experts * d * F bytes; MOE_EINVAL for
+ * an n_experts outside that range.
+ */
+MOE_API int moe_pack_weight_n(moe_handle h, const int8_t *w, int8_t *w_packed, int which, int n_experts,
+                              void *stream);
 
 /*
  * The tile shape and split chosen for T tokens (for tests and benchmarks):

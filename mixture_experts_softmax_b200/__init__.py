@@ -40,7 +40,7 @@ EXPORTS = (
     "moe_forward", "moe_forward_host", "moe_block_forward", "moe_get_routing", "moe_get_block_input",
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
     "moe_set_weight_layout", "moe_pack_weight", "moe_route_noalloc",
-    "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
+    "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_set_cta_pairs", "moe_pack_weight_n",
 )
 
 
@@ -77,10 +77,12 @@ def _load() -> ctypes.CDLL:
         "moe_plan": (I, [P, I, ctypes.POINTER(I), ctypes.POINTER(I)]),
         "moe_set_weight_layout": (I, [P, I]),
         "moe_pack_weight": (I, [P, P, P, I, P]),
+        "moe_pack_weight_n": (I, [P, P, P, I, I, P]),
         "moe_route_noalloc": (I, [I, I, P, P, P, P, P, P, P, P]),
         "moe_ep_dispatch": (I, [P, I, P, P, P, P, P]),
         "moe_ep_experts": (I, [P, I, I, P, P, P, P, P, P, P, P, P, P]),
         "moe_ep_combine": (I, [P, I, P, P, P]),
+        "moe_set_cta_pairs": (I, [P, I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -200,6 +202,11 @@ def moe_get_kernel_times(h):
     return rc, {KERNEL_NAMES[i]: (ms[i], cnt[i]) for i in range(n)}
 
 
+def moe_set_cta_pairs(h, on: bool) -> int:
+    """Up-projection of 128-route tiles on CTA pairs (default) or one CTA per tile."""
+    return _lib.moe_set_cta_pairs(h, 1 if on else 0)
+
+
 def moe_set_weight_layout(h, layout: int) -> int:
     return _lib.moe_set_weight_layout(h, int(layout))
 
@@ -208,16 +215,21 @@ def moe_pack_weight(h, w, w_packed, which: int, stream=None) -> int:
     return _lib.moe_pack_weight(h, _ptr(w), _ptr(w_packed), int(which), _stream(stream))
 
 
+def moe_pack_weight_n(h, w, w_packed, which: int, n_experts: int, stream=None) -> int:
+    return _lib.moe_pack_weight_n(h, _ptr(w), _ptr(w_packed), int(which), int(n_experts), _stream(stream))
+
+
 def pack_layer(h, layer: dict, stream=None) -> dict:
     """A copy of `layer` with its three int8 weights rewritten to MOE_LAYOUT_PACKED
-    (new device buffers; scales and router weight shared with `layer`)."""
+    (new device buffers; scales and router weight shared with `layer`).  The weights may
+    hold fewer experts than the handle (an expert-parallel rank's share)."""
     import torch
     out = dict(layer)
     for key, which in (("wl", 0), ("wv", 0), ("w1", 1)):
         w = layer[key]
         E, a, b = w.shape
         p = torch.empty((E, b, a), dtype=torch.int8, device=w.device)
-        check(moe_pack_weight(h, w, p, which, stream), "moe_pack_weight")
+        check(moe_pack_weight_n(h, w, p, which, E, stream), "moe_pack_weight_n")
         out[key] = p
     return out
 

@@ -75,6 +75,7 @@ struct moe_ctx {
     int kblock = 0;                  // scale format: 0 per output channel, kScaleBlock per block
     long long timeout_ns = 2000000000LL;
     int layout = MOE_LAYOUT_IN_OUT;
+    bool cta_pairs = true;           // up-projection of 128-route tiles on CTA pairs (packed layout)
 
     // profiling
     bool prof = false;
@@ -392,6 +393,9 @@ int check_weights(const moe_ctx *h, const float *router_w, const int8_t *w_lin, 
     return MOE_OK;
 }
 
+cudaError_t launch_up(moe_ctx *h, int bn, const CUtensorMap &m_wl, const CUtensorMap &m_wv, const CUtensorMap &m_b,
+                      const GemmArgs &up, cudaStream_t s);
+
 // the layer on x (device, bf16 [T, d]); result into `out` (plain) or added into h_io (residual block)
 int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int8_t *w_lin, const void *s_lin,
               const int8_t *w_v, const void *s_v, const int8_t *w_1, const void *s_1, void *out, void *h_io,
@@ -477,10 +481,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
         up.part = static_cast<float *>(h->b_part.ptr);
         up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
     }
-    if (timed(h, K_UP, s, [&] {
-            return ts ? launch_gemm_up_ts(bn, m_wl, m_wv, *m_b, up, h->num_sms, s)
-                      : launch_gemm_up(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s);
-        }) != cudaSuccess)
+    if (timed(h, K_UP, s, [&] { return launch_up(h, bn, m_wl, m_wv, ts ? *m_b : *m_xp, up, s); }) != cudaSuccess)
         return MOE_ECUDA;
 
     GemmArgs dn = up;
@@ -521,6 +522,21 @@ int begin_call(moe_ctx *h, int T, cudaStream_t s)
     h->last_stream = s;
     h->used = true;
     return MOE_OK;
+}
+
+// the up-projection launch of the handle's layout and plan: CTA pairs for 128-route tiles of the
+// packed layout when the device can hold a wave of them, else one CTA per tile
+cudaError_t launch_up(moe_ctx *h, int bn, const CUtensorMap &m_wl, const CUtensorMap &m_wv, const CUtensorMap &m_b,
+                      const GemmArgs &up, cudaStream_t s)
+{
+    if (h->layout != MOE_LAYOUT_PACKED) return launch_gemm_up(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
+    if (h->cta_pairs && bn == 128 && !up.gather && h->F % 256 == 0) {
+        const int grid = gemm_up_pair_grid(h->num_sms);
+        const CUtensorMap *xp64, *h64;
+        if (grid >= 2 && act_maps(h, 64, &xp64, &h64) == MOE_OK)
+            return launch_gemm_up_pair(m_wl, m_wv, *xp64, up, grid, s);
+    }
+    return launch_gemm_up_ts(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
 }
 
 // ---- expert parallelism (device steps; the exchange between ranks is the caller's) ----------
@@ -651,10 +667,7 @@ int run_ep_experts(moe_ctx *h, int n_src, int E_local, const int32_t *counts, in
         up.part = static_cast<float *>(h->b_part.ptr);
         up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
     }
-    if (timed(h, K_UP, s, [&] {
-            return ts ? launch_gemm_up_ts(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s)
-                      : launch_gemm_up(bn, m_wl, m_wv, *m_xp, up, h->num_sms, s);
-        }) != cudaSuccess)
+    if (timed(h, K_UP, s, [&] { return launch_up(h, bn, m_wl, m_wv, *m_xp, up, s); }) != cudaSuccess)
         return MOE_ECUDA;
     GemmArgs dn = up;
     dn.M = h->d;
@@ -764,6 +777,13 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns)
     return MOE_OK;
 }
 
+MOE_API int moe_set_cta_pairs(moe_handle h, int on)
+{
+    if (!h) return MOE_EINVAL;
+    h->cta_pairs = on != 0;
+    return MOE_OK;
+}
+
 MOE_API int moe_set_weight_layout(moe_handle h, int layout)
 {
     if (!h || (layout != MOE_LAYOUT_IN_OUT && layout != MOE_LAYOUT_PACKED)) return MOE_EINVAL;
@@ -771,18 +791,25 @@ MOE_API int moe_set_weight_layout(moe_handle h, int layout)
     return MOE_OK;
 }
 
-MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream)
+MOE_API int moe_pack_weight_n(moe_handle h, const int8_t *w, int8_t *w_packed, int which, int n_experts,
+                              void *stream)
 {
     if (!h || !w || !w_packed || !aligned16(w) || !aligned16(w_packed)) return MOE_EINVAL;
     if (which != 0 && which != 1) return MOE_EINVAL;
-    const size_t bytes = static_cast<size_t>(h->E) * h->d * h->F;
+    if (n_experts < 1 || n_experts > h->E) return MOE_EINVAL;
+    const size_t bytes = static_cast<size_t>(n_experts) * h->d * h->F;
     if (overlaps(w, bytes, w_packed, bytes)) return MOE_EINVAL;
     int rc = ensure_device(h);
     if (rc != MOE_OK) return rc;
     const int K = which == 0 ? h->d : h->F, M = which == 0 ? h->F : h->d;
-    return launch_transpose_i8(w, w_packed, h->E, K, M, static_cast<cudaStream_t>(stream)) == cudaSuccess
+    return launch_transpose_i8(w, w_packed, n_experts, K, M, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? MOE_OK
                : MOE_ECUDA;
+}
+
+MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream)
+{
+    return moe_pack_weight_n(h, w, w_packed, which, h ? h->E : 0, stream);
 }
 
 MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits)

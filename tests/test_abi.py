@@ -144,3 +144,17 @@ def test_block_input_needs_a_block_forward(m):
         assert m.moe_get_block_input(None, 1 << 20, 0) == m.MOE_EINVAL
     finally:
         m.moe_destroy(h)
+
+
+def test_pack_weight_n_checks_the_expert_count(m):
+    """An expert-parallel rank packs its own experts: the count must lie in 1 .. E (checked on
+    the host before any device work)."""
+    rc, h = m.moe_create(256, 512, 8, 2)
+    assert rc == m.MOE_OK
+    try:
+        A, B = 1 << 20, 1 << 30   # aligned, far apart: the count check comes first
+        assert m.moe_pack_weight_n(h, A, B, 0, 0, 0) == m.MOE_EINVAL
+        assert m.moe_pack_weight_n(h, A, B, 0, 9, 0) == m.MOE_EINVAL
+        assert m.moe_pack_weight_n(h, A, B, 2, 4, 0) == m.MOE_EINVAL
+    finally:
+        m.moe_destroy(h)

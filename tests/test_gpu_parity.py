@@ -265,6 +265,28 @@ def test_block_scales(m, tiny_inputs, tiny_handle, T):
     parity.check_output(run, layer_cpu, x_cpu, range(T), near)
 
 
+@pytest.mark.parametrize("T", [65, 300, 1000])
+def test_cta_pairs_match_single_cta(m, tiny_inputs, tiny_handle, T):
+    """The up-projection of 128-route tiles on CTA pairs (the default for the packed layout)
+    and on one CTA per tile give the same bits, and both match the oracle; the API layout
+    ignores the switch."""
+    h, layer, layout = tiny_handle
+    m.check(m.moe_set_router_bias(h, None))
+    m.check(m.moe_set_padding_mask(h, None))
+    x = tiny_inputs.x[:T].cuda()
+    try:
+        m.check(m.moe_set_cta_pairs(h, False))
+        single = parity.Run(h, x, layer)
+        m.check(m.moe_set_cta_pairs(h, True))
+        paired = parity.Run(h, x, layer)
+    finally:
+        m.check(m.moe_set_cta_pairs(h, True))
+    assert torch.equal(paired.out_h, single.out_h)
+    ref = oracle.route(tiny_inputs.x[:T], tiny_inputs.layers[0]["router_w"])
+    near = parity.check_routing(paired, ref, 8)
+    parity.check_output(paired, tiny_inputs.layers[0], tiny_inputs.x[:T], range(T), near)
+
+
 def test_pack_weight_is_a_transpose(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
@@ -274,6 +296,12 @@ def test_pack_weight_is_a_transpose(m, tiny_handle):
         m.check(m.moe_pack_weight(h, w, p, which))
         torch.cuda.synchronize()
         assert torch.equal(p, w.transpose(1, 2))
+        # a rank's share of the experts: exactly its bytes are read and written
+        part = w[2:5].contiguous()
+        guard = torch.full((4, shape[2], shape[1]), 7, dtype=torch.int8, device="cuda")
+        m.check(m.moe_pack_weight_n(h, part, guard, which, 3))
+        torch.cuda.synchronize()
+        assert torch.equal(guard[:3], part.transpose(1, 2)) and bool((guard[3] == 7).all())
 
 
 def test_tiny_maximum_token_count(m, tiny_handle):
@@ -342,6 +370,25 @@ def test_decode_T8_rerun_bit_identical(m, grok_handle):
     b = parity.Run(h, x, layer)
     assert torch.equal(a.out_h, b.out_h)
     assert np.array_equal(a.perm_h, b.perm_h) and np.array_equal(a.gate_h, b.gate_h)
+
+
+def test_prefill_cta_pairs_match_single_cta(m, grok_handle):
+    """Grok-1 shape, T = 2048 (every expert several 128-route tiles): CTA pairs and single CTAs
+    give the same output bits."""
+    h, layer, layout = grok_handle
+    if layout != m.MOE_LAYOUT_PACKED:
+        pytest.skip("CTA pairs serve the packed layout")
+    g = moe_synth.generator(41, "cuda")
+    x = moe_synth.draw_tokens(2048, 6144, g, "cuda")
+    m.check(m.moe_set_router_bias(h, None))
+    try:
+        m.check(m.moe_set_cta_pairs(h, False))
+        single = parity.Run(h, x, layer)
+        m.check(m.moe_set_cta_pairs(h, True))
+        paired = parity.Run(h, x, layer)
+    finally:
+        m.check(m.moe_set_cta_pairs(h, True))
+    assert torch.equal(paired.out_h, single.out_h)
 
 
 @pytest.mark.parametrize("name,T", [("prefill", 8192), ("skewed", 4096)])
