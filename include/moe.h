@@ -249,13 +249,16 @@ MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
 MOE_API int moe_set_weight_layout(moe_handle h, int layout);
 
 /*
- * Up-projection of large batches (128-route tiles, MOE_LAYOUT_PACKED, ffn a multiple of
- * 256) on CTA pairs: one tcgen05 MMA of 256 output features spans the two SMs of a
- * two-CTA cluster, each SM converting its 128 features' weights and holding half of the
- * 128 routes' activations, which halves the activation traffic through each SM's shared
- * memory.  on = 1 (the default) uses pairs where the device can run a full wave of them;
- * on = 0 keeps one CTA per tile.  Both compute the same sums (same order along the
- * reduction), so the results are the same.  Returns MOE_EINVAL for a NULL handle.
+ * The grouped GEMMs of large batches (128-route plans, MOE_LAYOUT_PACKED) on CTA pairs: one
+ * tcgen05 MMA of 256 output features spans the two SMs of a two-CTA cluster, each SM
+ * converting its 128 features' weights and holding half of the tile's routes' activations,
+ * which halves the activation traffic through each SM's shared memory.  The up-projection
+ * (ffn a multiple of 256) takes tiles of 128 routes, the down-projection (d a multiple of 256)
+ * tiles of 256.  on = 1 (the default) uses pairs where the device can run a full wave of
+ * them; on = 0 keeps one CTA per tile.  Both add the same products in the same order along
+ * the reduction, except that one CTA per tile cuts the tiles of a last, partial wave into
+ * K pieces added afterwards; outside such tiles the results are bit-identical.  Returns
+ * MOE_EINVAL for a NULL handle.
  */
 MOE_API int moe_set_cta_pairs(moe_handle h, int on);
 

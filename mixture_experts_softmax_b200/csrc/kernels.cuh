@@ -152,8 +152,13 @@ cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &w1, const CUtensorMap
 // gathered-rows map with 64-row boxes; a.M a multiple of 256; grid = gemm_up_pair_grid() CTAs
 cudaError_t launch_gemm_up_pair(const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
                                 const GemmArgs &a, int grid, cudaStream_t s);
+// the down-projection of 256-route tiles (two 128-row segments) on CTA pairs: h is the
+// H map with 128-row boxes; a.M a multiple of 256
+cudaError_t launch_gemm_down_pair(const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a, int grid,
+                                  cudaStream_t s);
 // CTAs of a full wave of pairs on this device (0 if pairs cannot be launched)
 int gemm_up_pair_grid(int num_sms);
+int gemm_down_pair_grid(int num_sms);
 // reduction elements per pipeline stage of the TMEM-operand GEMM (up- or down-projection, tile width bn)
 int gemm_ts_kstage(bool up, int bn);
 // out[e, m, k] = in[e, k, m] for E int8 [K, M] matrices (K, M multiples of 64)

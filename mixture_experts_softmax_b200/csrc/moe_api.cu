@@ -395,6 +395,8 @@ int check_weights(const moe_ctx *h, const float *router_w, const int8_t *w_lin, 
 
 cudaError_t launch_up(moe_ctx *h, int bn, const CUtensorMap &m_wl, const CUtensorMap &m_wv, const CUtensorMap &m_b,
                       const GemmArgs &up, cudaStream_t s);
+cudaError_t launch_down(moe_ctx *h, int bn, const CUtensorMap &m_w1, const CUtensorMap &m_h, const GemmArgs &dn,
+                        cudaStream_t s);
 
 // the layer on x (device, bf16 [T, d]); result into `out` (plain) or added into h_io (residual block)
 int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int8_t *w_lin, const void *s_lin,
@@ -494,10 +496,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     dn.s1 = nullptr;
     dn.h = nullptr;
     dn.slots = static_cast<float *>(h->b_slots.ptr);
-    if (timed(h, K_DOWN, s, [&] {
-            return ts ? launch_gemm_down_ts(bn, m_w1, *m_h, dn, h->num_sms, s)
-                      : launch_gemm_down(bn, m_w1, *m_h, dn, h->num_sms, s);
-        }) != cudaSuccess)
+    if (timed(h, K_DOWN, s, [&] { return launch_down(h, bn, m_w1, *m_h, dn, s); }) != cudaSuccess)
         return MOE_ECUDA;
 
     h->last_block_T = g_pre ? T : -1;
@@ -537,6 +536,18 @@ cudaError_t launch_up(moe_ctx *h, int bn, const CUtensorMap &m_wl, const CUtenso
             return launch_gemm_up_pair(m_wl, m_wv, *xp64, up, grid, s);
     }
     return launch_gemm_up_ts(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
+}
+
+// the down-projection launch: CTA pairs for the packed layout's 256-route tiles (bn = 128)
+cudaError_t launch_down(moe_ctx *h, int bn, const CUtensorMap &m_w1, const CUtensorMap &m_h, const GemmArgs &dn,
+                        cudaStream_t s)
+{
+    if (h->layout != MOE_LAYOUT_PACKED) return launch_gemm_down(bn, m_w1, m_h, dn, h->num_sms, s);
+    if (h->cta_pairs && bn == 128 && h->d % 256 == 0) {
+        const int grid = gemm_down_pair_grid(h->num_sms);
+        if (grid >= 2) return launch_gemm_down_pair(m_w1, m_h, dn, grid, s);
+    }
+    return launch_gemm_down_ts(bn, m_w1, m_h, dn, h->num_sms, s);
 }
 
 // ---- expert parallelism (device steps; the exchange between ranks is the caller's) ----------
@@ -679,10 +690,7 @@ int run_ep_experts(moe_ctx *h, int n_src, int E_local, const int32_t *counts, in
     dn.h = nullptr;
     // one split: route id i lands in row i of [Tp, 2, d] = y_rows itself
     dn.slots = splits == 1 ? y_rows : static_cast<float *>(h->b_slots.ptr);
-    if (timed(h, K_DOWN, s, [&] {
-            return ts ? launch_gemm_down_ts(bn, m_w1, *m_h, dn, h->num_sms, s)
-                      : launch_gemm_down(bn, m_w1, *m_h, dn, h->num_sms, s);
-        }) != cudaSuccess)
+    if (timed(h, K_DOWN, s, [&] { return launch_down(h, bn, m_w1, *m_h, dn, s); }) != cudaSuccess)
         return MOE_ECUDA;
     if (splits > 1 && timed(h, K_COMBINE, s, [&] {
             return launch_ep_split_sum(R, h->d, splits, static_cast<size_t>(Tp) * 2 * h->d,
