@@ -68,8 +68,10 @@ def parse(argv=None):
                    help="weight scale format: 0 per output channel, 128 per block of 128 inputs (packed layout)")
     p.add_argument("--layout", choices=("packed", "in_out"), default="packed",
                    help="weight layout: packed = tiles written once at load (TMEM path); in_out = as drawn")
-    p.add_argument("--no-cta-pairs", action="store_true",
-                   help="up-projection of 128-route tiles on one CTA per tile instead of CTA pairs (comparison)")
+    p.add_argument("--cta-pairs", type=int, choices=(0, 1, 2), default=None,
+                   help="GEMMs on CTA pairs: 0 never, 1 for 128-route plans (library default), 2 also small batches")
+    p.add_argument("--no-cta-pairs", dest="cta_pairs", action="store_const", const=0,
+                   help="the same as --cta-pairs 0")
     p.add_argument("--parallel", choices=("replicas", "ep"), default="replicas",
                    help="several GPUs: independent replicas (default), or experts spread over the ranks "
                         "(each rank E/N experts and its own tokens; all-to-all exchanges over NCCL)")
@@ -317,7 +319,8 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
     stream = torch.cuda.current_stream(dev)
 
     h = moe.MoELayer(w.d, w.F, w.E, w.k)
-    moe.check(moe.moe_set_cta_pairs(h.h, not args.no_cta_pairs))
+    if args.cta_pairs is not None:
+        moe.check(moe.moe_set_cta_pairs(h.h, args.cta_pairs))
     moe.check(moe.moe_set_router_bias(h.h, inp.bias))
     moe.check(moe.moe_set_scale_block(h.h, args.scale_block))
     if layout == "packed":
@@ -389,7 +392,7 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
                                  ", layout " + layout +
                                  (" (packed once at load, untimed)" if layout == "packed" else " (as drawn)"),
                       "parallelism": f"replicas x{world}", "tile_routes": moe.moe_plan(h.h, T)[1],
-                      "cta_pairs": not args.no_cta_pairs,
+                      "cta_pairs": "library default" if args.cta_pairs is None else args.cta_pairs,
                       "down_splits": moe.moe_plan(h.h, T)[2]},
            "clocks": clk}
 

@@ -249,18 +249,22 @@ MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
 MOE_API int moe_set_weight_layout(moe_handle h, int layout);
 
 /*
- * The grouped GEMMs of large batches (128-route plans, MOE_LAYOUT_PACKED) on CTA pairs: one
- * tcgen05 MMA of 256 output features spans the two SMs of a two-CTA cluster, each SM
- * converting its 128 features' weights and holding half of the tile's routes' activations,
- * which halves the activation traffic through each SM's shared memory.  The up-projection
- * (ffn a multiple of 256) takes tiles of 128 routes, the down-projection (d a multiple of 256)
- * tiles of 256.  on = 1 (the default) uses pairs where the device can run a full wave of
- * them; on = 0 keeps one CTA per tile.  Both add the same products in the same order along
- * the reduction, except that one CTA per tile cuts the tiles of a last, partial wave into
- * K pieces added afterwards; outside such tiles the results are bit-identical.  Returns
- * MOE_EINVAL for a NULL handle.
+ * The grouped GEMMs on CTA pairs (MOE_LAYOUT_PACKED, d and ffn multiples of 256): one tcgen05
+ * MMA of 256 output features spans the two SMs of a two-CTA cluster, each SM converting its
+ * 128 features' weights and holding half of the tile's routes' activations.  For large
+ * batches that halves the activation traffic through each SM's shared memory (the
+ * up-projection takes tiles of 128 routes, the down-projection of 256); for small batches each
+ * MMA, of few columns, covers twice the features (tiles of 32 routes).
+ *   mode 0  one CTA per tile everywhere (the default: on a B200 the pairs measured slower);
+ *   mode 1  pairs for plans of 128-route tiles (T > 64);
+ *   mode 2  pairs also for T <= 32 (32-route tiles).
+ * Pairs run only where the device can hold a full wave of them.  Both paths add the same
+ * products in the same order along the reduction, except where the tiles of a last, partial
+ * wave are cut into K pieces added afterwards (each path cuts its own last wave); elsewhere
+ * the results are bit-identical.  The mode applies to later forwards (it also sets the tile
+ * width moe_plan reports).  Returns MOE_EINVAL for a NULL handle or another mode.
  */
-MOE_API int moe_set_cta_pairs(moe_handle h, int on);
+MOE_API int moe_set_cta_pairs(moe_handle h, int mode);
 
 /*
  * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT to MOE_LAYOUT_PACKED

@@ -202,9 +202,14 @@ def moe_get_kernel_times(h):
     return rc, {KERNEL_NAMES[i]: (ms[i], cnt[i]) for i in range(n)}
 
 
-def moe_set_cta_pairs(h, on: bool) -> int:
-    """Up-projection of 128-route tiles on CTA pairs (default) or one CTA per tile."""
-    return _lib.moe_set_cta_pairs(h, 1 if on else 0)
+MOE_PAIRS_OFF = 0      # one CTA per GEMM tile (the default)
+MOE_PAIRS_LARGE = 1    # CTA pairs for 128-route plans
+MOE_PAIRS_ALL = 2      # CTA pairs also for small batches (32-route plans)
+
+
+def moe_set_cta_pairs(h, mode: int) -> int:
+    """GEMMs on CTA pairs: MOE_PAIRS_OFF (default), MOE_PAIRS_LARGE or MOE_PAIRS_ALL."""
+    return _lib.moe_set_cta_pairs(h, int(mode))
 
 
 def moe_set_weight_layout(h, layout: int) -> int:

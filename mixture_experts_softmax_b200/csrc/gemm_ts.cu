@@ -454,8 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = it % C::NDB;
             const uint32_t aph = (it / C::NDB) & 1;
             PS_NOW(t0);
-            const bool ok = __all_sync(0xffffffffu, w.wait(acc_full(b), aph, 6));
-            if (!ok) break;
+            w.wait(acc_full(b), aph, 6);   // a wait that gives up sets the CTA's abort flag
+            // one decision for all epilogue warps: a piece's epilogue meets at a named barrier,
+            // so no warp may leave the loop while the others go on
+            epilogue_sync();
+            if (*abort_flag) break;
             PS_ADD(c_ewait, t0);
             PS_NOW(t1);
             tc_fence_after();

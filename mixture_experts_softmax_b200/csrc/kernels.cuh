@@ -148,17 +148,18 @@ cudaError_t launch_gemm_up_ts(int bn, const CUtensorMap &wl, const CUtensorMap &
                               const GemmArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_gemm_down_ts(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a,
                                 int grid, cudaStream_t s);
-// the up-projection of 128-route tiles on CTA pairs (M = 256 per MMA across two SMs): xp is the
-// gathered-rows map with 64-row boxes; a.M a multiple of 256; grid = gemm_up_pair_grid() CTAs
-cudaError_t launch_gemm_up_pair(const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
-                                const GemmArgs &a, int grid, cudaStream_t s);
-// the down-projection of 256-route tiles (two 128-row segments) on CTA pairs: h is the
-// H map with 128-row boxes; a.M a multiple of 256
-cudaError_t launch_gemm_down_pair(const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a, int grid,
+// The GEMMs of a plan with tile width bn on CTA pairs (M = 256 per MMA across two SMs), for
+// bn = 32 (tiles of 32 routes) and bn = 128 (up-projection tiles of 128 routes, down-projection
+// tiles of two 128-row segments).  gemm_pair_tn: routes per pair tile, 0 if bn has no pair
+// kernel; each CTA holds tn / 2 route rows, so the activation map (xp for the up-projection, or
+// the routed-rows map with a.gather; H for the down-projection) has boxes of tn / 2 rows.
+// gemm_pair_ready: the device can run a full wave of that kernel's pairs.  a.M a multiple of 256.
+int gemm_pair_tn(bool up, int bn);
+bool gemm_pair_ready(bool up, int bn, int num_sms);
+cudaError_t launch_gemm_up_pair(int bn, const CUtensorMap &wl, const CUtensorMap &wv, const CUtensorMap &xp,
+                                const GemmArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_down_pair(int bn, const CUtensorMap &w1, const CUtensorMap &h, const GemmArgs &a, int num_sms,
                                   cudaStream_t s);
-// CTAs of a full wave of pairs on this device (0 if pairs cannot be launched)
-int gemm_up_pair_grid(int num_sms);
-int gemm_down_pair_grid(int num_sms);
 // reduction elements per pipeline stage of the TMEM-operand GEMM (up- or down-projection, tile width bn)
 int gemm_ts_kstage(bool up, int bn);
 // out[e, m, k] = in[e, k, m] for E int8 [K, M] matrices (K, M multiples of 64)

@@ -75,7 +75,7 @@ struct moe_ctx {
     int kblock = 0;                  // scale format: 0 per output channel, kScaleBlock per block
     long long timeout_ns = 2000000000LL;
     int layout = MOE_LAYOUT_IN_OUT;
-    bool cta_pairs = true;           // up-projection of 128-route tiles on CTA pairs (packed layout)
+    int cta_pairs = 0;               // GEMMs on CTA pairs (packed layout): 0 never, 1 large batches, 2 all
 
     // profiling
     bool prof = false;
@@ -91,12 +91,29 @@ constexpr int kCtlTickets = 64;     // first GEMM ticket
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int plan_bn(int T)
+// pair kernels for plans of tile width bn on this handle (both GEMMs must have one)
+bool pairs_for(const moe_ctx *h, int bn)
 {
-    if (T <= 16) return 16;
-    if (T <= 32) return 32;
-    if (T <= 64) return 64;
+    if (h->layout != MOE_LAYOUT_PACKED || h->d % 256 || h->F % 256) return false;
+    if (bn == 128) return h->cta_pairs >= 1;
+    if (bn == 32) return h->cta_pairs >= 2;
+    return false;
+}
+
+// routes per GEMM tile (the dispatch pads each expert's segment to it) for batches of about
+// `rows_per_expert` routes per expert; CTA pairs at small batches need 32-route tiles
+int plan_bn_rows(const moe_ctx *h, int rows_per_expert)
+{
+    if (rows_per_expert <= 16 && !pairs_for(h, 32)) return 16;
+    if (rows_per_expert <= 32) return 32;
+    if (rows_per_expert <= 64) return 64;
     return 128;
+}
+
+int plan_bn(const moe_ctx *h, int T)
+{
+    // by T: T <= 16 -> 16 (32 with small-batch pairs), <= 32 -> 32, <= 64 -> 64, else 128
+    return plan_bn_rows(h, T);
 }
 
 int bn_slot(int bn) { return bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3; }
@@ -404,7 +421,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
               const void *g_pre, const void *g_post, float eps, cudaStream_t s)
 {
     int rc;
-    const int bn = plan_bn(T);
+    const int bn = plan_bn(h, T);
     const int splits = plan_splits(h, T, bn);
     const RouteLayout L = route_layout(T, h->E);
     int *rw = static_cast<int *>(h->b_route.ptr);
@@ -516,36 +533,38 @@ int begin_call(moe_ctx *h, int T, cudaStream_t s)
         // work of the previous stream may still use the workspace
         if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
     }
-    const int bn = plan_bn(T);
+    const int bn = plan_bn(h, T);
     if ((rc = ensure_workspace(h, T, bn, plan_splits(h, T, bn))) != MOE_OK) return rc;
     h->last_stream = s;
     h->used = true;
     return MOE_OK;
 }
 
-// the up-projection launch of the handle's layout and plan: CTA pairs for 128-route tiles of the
-// packed layout when the device can hold a wave of them, else one CTA per tile
+// the up-projection launch of the handle's layout and plan: CTA pairs where the plan has them and
+// the device can hold a wave of them, else one CTA per tile.  m_b: the routed-rows map (one-row
+// boxes) when up.gather, else the gathered rows with bn-row boxes.
 cudaError_t launch_up(moe_ctx *h, int bn, const CUtensorMap &m_wl, const CUtensorMap &m_wv, const CUtensorMap &m_b,
                       const GemmArgs &up, cudaStream_t s)
 {
     if (h->layout != MOE_LAYOUT_PACKED) return launch_gemm_up(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
-    if (h->cta_pairs && bn == 128 && !up.gather && h->F % 256 == 0) {
-        const int grid = gemm_up_pair_grid(h->num_sms);
-        const CUtensorMap *xp64, *h64;
-        if (grid >= 2 && act_maps(h, 64, &xp64, &h64) == MOE_OK)
-            return launch_gemm_up_pair(m_wl, m_wv, *xp64, up, grid, s);
+    if (pairs_for(h, bn) && gemm_pair_ready(true, bn, h->num_sms) && gemm_pair_ready(false, bn, h->num_sms)) {
+        if (up.gather) return launch_gemm_up_pair(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
+        const CUtensorMap *xph, *hh;   // maps with boxes of half a pair tile
+        if (act_maps(h, gemm_pair_tn(true, bn) / 2, &xph, &hh) == MOE_OK)
+            return launch_gemm_up_pair(bn, m_wl, m_wv, *xph, up, h->num_sms, s);
     }
     return launch_gemm_up_ts(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
 }
 
-// the down-projection launch: CTA pairs for the packed layout's 256-route tiles (bn = 128)
+// the down-projection launch: CTA pairs where the plan has them (same rule as launch_up)
 cudaError_t launch_down(moe_ctx *h, int bn, const CUtensorMap &m_w1, const CUtensorMap &m_h, const GemmArgs &dn,
                         cudaStream_t s)
 {
     if (h->layout != MOE_LAYOUT_PACKED) return launch_gemm_down(bn, m_w1, m_h, dn, h->num_sms, s);
-    if (h->cta_pairs && bn == 128 && h->d % 256 == 0) {
-        const int grid = gemm_down_pair_grid(h->num_sms);
-        if (grid >= 2) return launch_gemm_down_pair(m_w1, m_h, dn, grid, s);
+    if (pairs_for(h, bn) && gemm_pair_ready(true, bn, h->num_sms) && gemm_pair_ready(false, bn, h->num_sms)) {
+        const CUtensorMap *xph, *hh;
+        if (act_maps(h, gemm_pair_tn(false, bn) / 2, &xph, &hh) == MOE_OK)
+            return launch_gemm_down_pair(bn, m_w1, *hh, dn, h->num_sms, s);
     }
     return launch_gemm_down_ts(bn, m_w1, m_h, dn, h->num_sms, s);
 }
@@ -613,7 +632,7 @@ int run_ep_experts(moe_ctx *h, int n_src, int E_local, const int32_t *counts, in
                    const int8_t *w_1, const void *s_1, float *y_rows, cudaStream_t s)
 {
     int rc;
-    const int bn = max_rows <= 16 ? 16 : max_rows <= 32 ? 32 : max_rows <= 64 ? 64 : 128;
+    const int bn = plan_bn_rows(h, max_rows);
     const int splits = splits_for(h, E_local, max_rows, bn);
     const int Tp = (R + 1) / 2;   // the down-projection's slots [splits, Tp, 2, d] hold rows [splits, 2 Tp, d]
     const int rows = ((R + E_local * (bn - 1)) + 127) / 128 * 128;
@@ -785,10 +804,10 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns)
     return MOE_OK;
 }
 
-MOE_API int moe_set_cta_pairs(moe_handle h, int on)
+MOE_API int moe_set_cta_pairs(moe_handle h, int mode)
 {
-    if (!h) return MOE_EINVAL;
-    h->cta_pairs = on != 0;
+    if (!h || mode < 0 || mode > 2) return MOE_EINVAL;
+    h->cta_pairs = mode;
     return MOE_OK;
 }
 
@@ -823,7 +842,7 @@ MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int
 MOE_API int moe_plan(moe_handle h, int T, int *bn, int *splits)
 {
     if (!h || T < 0 || T > MOE_MAX_TOKENS) return MOE_EINVAL;
-    const int b = plan_bn(T);
+    const int b = plan_bn(h, T);
     if (bn) *bn = b;
     if (splits) *splits = plan_splits(h, T, b);
     return MOE_OK;
