@@ -278,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const WorkList wl = a.part ? make_work_list(total, static_cast<int>(npairs), a.ksteps) : WorkList{total, 0, total};
     const WaiterC w{abort_flag, a.err, a.timeout_ns};
     const int SB = (UP ? 0 : 32) + (cta ? 16 : 0);   // first stats slot (instrumented builds)
+    (void)SB;
     PS_NOW(t_start);
 
     if (warp == kWarpTmaA) {
