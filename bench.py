@@ -68,8 +68,9 @@ def parse(argv=None):
                    help="weight scale format: 0 per output channel, 128 per block of 128 inputs (packed layout)")
     p.add_argument("--layout", choices=("packed", "in_out"), default="packed",
                    help="weight layout: packed = tiles written once at load (TMEM path); in_out = as drawn")
-    p.add_argument("--cta-pairs", type=int, choices=(0, 1, 2), default=None,
-                   help="GEMMs on CTA pairs: 0 never, 1 for 128-route plans (library default), 2 also small batches")
+    p.add_argument("--cta-pairs", type=int, choices=(0, 1, 2, 3), default=None,
+                   help="GEMMs on CTA pairs: 0 never, 1 the down-projection of 128-route plans (library default), "
+                        "2 both GEMMs of those plans, 3 also small batches")
     p.add_argument("--no-cta-pairs", dest="cta_pairs", action="store_const", const=0,
                    help="the same as --cta-pairs 0")
     p.add_argument("--parallel", choices=("replicas", "ep"), default="replicas",

@@ -255,14 +255,19 @@ MOE_API int moe_set_weight_layout(moe_handle h, int layout);
  * batches that halves the activation traffic through each SM's shared memory (the
  * up-projection takes tiles of 128 routes, the down-projection of 256); for small batches each
  * MMA, of few columns, covers twice the features (tiles of 32 routes).
- *   mode 0  one CTA per tile everywhere (the default: on a B200 the pairs measured slower);
- *   mode 1  pairs for plans of 128-route tiles (T > 64);
- *   mode 2  pairs also for T <= 32 (32-route tiles).
+ *   mode 0  one CTA per tile everywhere;
+ *   mode 1  pairs for the down-projection of plans of 128-route tiles (T > 64), the default:
+ *           on a B200 it ran 12% faster than one CTA per tile at T = 8192;
+ *   mode 2  pairs for both GEMMs of those plans (the up-projection measured slower on pairs:
+ *           its two-stage TMEM operand ring leaves the cross-SM signals too little slack);
+ *   mode 3  pairs also for both GEMMs of T <= 32 (32-route tiles; there the int8 -> bf16
+ *           conversion, which pairs do not shorten, limits both paths).
  * Pairs run only where the device can hold a full wave of them.  Both paths add the same
  * products in the same order along the reduction, except where the tiles of a last, partial
  * wave are cut into K pieces added afterwards (each path cuts its own last wave); elsewhere
  * the results are bit-identical.  The mode applies to later forwards (it also sets the tile
- * width moe_plan reports).  Returns MOE_EINVAL for a NULL handle or another mode.
+ * width moe_plan reports: 32 from T = 1 with mode 3).  Returns MOE_EINVAL for a NULL handle or
+ * another mode.
  */
 MOE_API int moe_set_cta_pairs(moe_handle h, int mode);
 

@@ -202,13 +202,14 @@ def moe_get_kernel_times(h):
     return rc, {KERNEL_NAMES[i]: (ms[i], cnt[i]) for i in range(n)}
 
 
-MOE_PAIRS_OFF = 0      # one CTA per GEMM tile (the default)
-MOE_PAIRS_LARGE = 1    # CTA pairs for 128-route plans
-MOE_PAIRS_ALL = 2      # CTA pairs also for small batches (32-route plans)
+MOE_PAIRS_OFF = 0          # one CTA per GEMM tile
+MOE_PAIRS_LARGE_DOWN = 1   # CTA pairs for the down-projection of 128-route plans (the default)
+MOE_PAIRS_LARGE = 2        # CTA pairs for both GEMMs of 128-route plans
+MOE_PAIRS_ALL = 3          # CTA pairs also for small batches (32-route plans)
 
 
 def moe_set_cta_pairs(h, mode: int) -> int:
-    """GEMMs on CTA pairs: MOE_PAIRS_OFF (default), MOE_PAIRS_LARGE or MOE_PAIRS_ALL."""
+    """GEMMs on CTA pairs: one of the MOE_PAIRS_* modes (MOE_PAIRS_LARGE_DOWN by default)."""
     return _lib.moe_set_cta_pairs(h, int(mode))
 
 

@@ -75,7 +75,9 @@ struct moe_ctx {
     int kblock = 0;                  // scale format: 0 per output channel, kScaleBlock per block
     long long timeout_ns = 2000000000LL;
     int layout = MOE_LAYOUT_IN_OUT;
-    int cta_pairs = 0;               // GEMMs on CTA pairs (packed layout): 0 never, 1 large batches, 2 all
+    // GEMMs on CTA pairs (packed layout): 0 never, 1 the down-projection of 128-route plans,
+    // 2 both GEMMs of 128-route plans, 3 also both GEMMs of 32-route plans
+    int cta_pairs = 1;
 
     // profiling
     bool prof = false;
@@ -91,12 +93,12 @@ constexpr int kCtlTickets = 64;     // first GEMM ticket
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// pair kernels for plans of tile width bn on this handle (both GEMMs must have one)
-bool pairs_for(const moe_ctx *h, int bn)
+// the up- (up = true) or down-projection of plans of tile width bn on CTA pairs on this handle
+bool pairs_for(const moe_ctx *h, int bn, bool up)
 {
     if (h->layout != MOE_LAYOUT_PACKED || h->d % 256 || h->F % 256) return false;
-    if (bn == 128) return h->cta_pairs >= 1;
-    if (bn == 32) return h->cta_pairs >= 2;
+    if (bn == 128) return h->cta_pairs >= (up ? 2 : 1);
+    if (bn == 32) return h->cta_pairs >= 3;
     return false;
 }
 
@@ -104,7 +106,7 @@ bool pairs_for(const moe_ctx *h, int bn)
 // `rows_per_expert` routes per expert; CTA pairs at small batches need 32-route tiles
 int plan_bn_rows(const moe_ctx *h, int rows_per_expert)
 {
-    if (rows_per_expert <= 16 && !pairs_for(h, 32)) return 16;
+    if (rows_per_expert <= 16 && !pairs_for(h, 32, true)) return 16;
     if (rows_per_expert <= 32) return 32;
     if (rows_per_expert <= 64) return 64;
     return 128;
@@ -547,7 +549,7 @@ cudaError_t launch_up(moe_ctx *h, int bn, const CUtensorMap &m_wl, const CUtenso
                       const GemmArgs &up, cudaStream_t s)
 {
     if (h->layout != MOE_LAYOUT_PACKED) return launch_gemm_up(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
-    if (pairs_for(h, bn) && gemm_pair_ready(true, bn, h->num_sms) && gemm_pair_ready(false, bn, h->num_sms)) {
+    if (pairs_for(h, bn, true) && gemm_pair_ready(true, bn, h->num_sms)) {
         if (up.gather) return launch_gemm_up_pair(bn, m_wl, m_wv, m_b, up, h->num_sms, s);
         const CUtensorMap *xph, *hh;   // maps with boxes of half a pair tile
         if (act_maps(h, gemm_pair_tn(true, bn) / 2, &xph, &hh) == MOE_OK)
@@ -561,7 +563,7 @@ cudaError_t launch_down(moe_ctx *h, int bn, const CUtensorMap &m_w1, const CUten
                         cudaStream_t s)
 {
     if (h->layout != MOE_LAYOUT_PACKED) return launch_gemm_down(bn, m_w1, m_h, dn, h->num_sms, s);
-    if (pairs_for(h, bn) && gemm_pair_ready(true, bn, h->num_sms) && gemm_pair_ready(false, bn, h->num_sms)) {
+    if (pairs_for(h, bn, false) && gemm_pair_ready(false, bn, h->num_sms)) {
         const CUtensorMap *xph, *hh;
         if (act_maps(h, gemm_pair_tn(false, bn) / 2, &xph, &hh) == MOE_OK)
             return launch_gemm_down_pair(bn, m_w1, *hh, dn, h->num_sms, s);
@@ -806,7 +808,7 @@ MOE_API int moe_set_timeout(moe_handle h, long long ns)
 
 MOE_API int moe_set_cta_pairs(moe_handle h, int mode)
 {
-    if (!h || mode < 0 || mode > 2) return MOE_EINVAL;
+    if (!h || mode < 0 || mode > 3) return MOE_EINVAL;
     h->cta_pairs = mode;
     return MOE_OK;
 }

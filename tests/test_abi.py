@@ -158,3 +158,16 @@ def test_pack_weight_n_checks_the_expert_count(m):
         assert m.moe_pack_weight_n(h, A, B, 2, 4, 0) == m.MOE_EINVAL
     finally:
         m.moe_destroy(h)
+
+
+def test_cta_pairs_modes(m):
+    rc, h = m.moe_create(256, 512, 8, 2)
+    assert rc == m.MOE_OK
+    try:
+        for mode in (m.MOE_PAIRS_OFF, m.MOE_PAIRS_LARGE_DOWN, m.MOE_PAIRS_LARGE, m.MOE_PAIRS_ALL):
+            assert m.moe_set_cta_pairs(h, mode) == m.MOE_OK
+        assert m.moe_set_cta_pairs(h, 4) == m.MOE_EINVAL
+        assert m.moe_set_cta_pairs(h, -1) == m.MOE_EINVAL
+        assert m.moe_set_cta_pairs(None, 1) == m.MOE_EINVAL
+    finally:
+        m.moe_destroy(h)

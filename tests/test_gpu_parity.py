@@ -265,7 +265,7 @@ def test_block_scales(m, tiny_inputs, tiny_handle, T):
     parity.check_output(run, layer_cpu, x_cpu, range(T), near)
 
 
-@pytest.mark.parametrize("T,mode", [(65, 1), (300, 1), (1000, 1), (1, 2), (8, 2), (17, 2), (32, 2)])
+@pytest.mark.parametrize("T,mode", [(65, 1), (300, 2), (1000, 2), (1, 3), (8, 3), (17, 3), (32, 3)])
 def test_cta_pairs_match_single_cta(m, tiny_inputs, tiny_handle, T, mode):
     """The GEMMs of 128-route plans on CTA pairs (the default for the packed layout) and on one
     CTA per tile give the same bits (these sizes have no last-wave pieces), and both match the
@@ -280,7 +280,7 @@ def test_cta_pairs_match_single_cta(m, tiny_inputs, tiny_handle, T, mode):
         m.check(m.moe_set_cta_pairs(h, mode))
         paired = parity.Run(h, x, layer)
     finally:
-        m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_OFF))
+        m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_LARGE_DOWN))
     assert torch.equal(paired.out_h, single.out_h)
     ref = oracle.route(tiny_inputs.x[:T], tiny_inputs.layers[0]["router_w"])
     near = parity.check_routing(paired, ref, 8)
@@ -372,7 +372,7 @@ def test_decode_T8_rerun_bit_identical(m, grok_handle):
     assert np.array_equal(a.perm_h, b.perm_h) and np.array_equal(a.gate_h, b.gate_h)
 
 
-@pytest.mark.parametrize("T,mode", [(2048, 1), (8, 2), (32, 2)])
+@pytest.mark.parametrize("T,mode", [(2048, 2), (8, 3), (32, 3)])
 def test_grok_cta_pairs_match_single_cta(m, grok_handle, grok_layer, T, mode):
     """Grok-1 shape: T = 2048 (every expert several 128-route tiles) and the decode sizes
     T = 8, 32 (32-route pair tiles, K-split down-projection, last-wave pieces, rows gathered
@@ -391,14 +391,14 @@ def test_grok_cta_pairs_match_single_cta(m, grok_handle, grok_layer, T, mode):
         m.check(m.moe_set_cta_pairs(h, mode))
         paired = parity.Run(h, x, layer)
     finally:
-        m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_OFF))
+        m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_LARGE_DOWN))
     a, b = paired.out_h.to(torch.float64), single.out_h.to(torch.float64)
     assert (a - b).abs().max() <= 2e-3 * b.abs().max()
     x_cpu = x.cpu()
     ref = oracle.route(x_cpu, layer_cpu["router_w"])
     near = parity.check_routing(paired, ref, 8)
     parity.check_output(paired, layer_cpu, x_cpu, parity.sample_tokens(paired, T, 32), near)
-    again = parity.Run(h, x, layer) if mode == 1 else None
+    again = parity.Run(h, x, layer) if mode == 2 else None
     if again is not None:
         assert torch.equal(again.out_h, paired.out_h)
 
@@ -437,12 +437,12 @@ def test_wide_tiles_odd_segments_and_pieces(m, grok_handle, grok_layer, pairs):
     g = moe_synth.generator(23, "cuda")
     x = moe_synth.draw_tokens(T, 6144, g, "cuda")
     bias = torch.tensor([100.0, 100.0, 0, 0, 0, 0, 0, 0])
-    m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_LARGE if pairs else m.MOE_PAIRS_OFF))
+    m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_LARGE_DOWN if pairs else m.MOE_PAIRS_OFF))
     try:
         run = parity.Run(h, x, layer, bias.cuda())
         again = parity.Run(h, x, layer, bias.cuda())     # a fixed summation order: same bits
     finally:
-        m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_OFF))
+        m.check(m.moe_set_cta_pairs(h, m.MOE_PAIRS_LARGE_DOWN))
     assert torch.equal(again.out_h, run.out_h)
     assert run.offsets_h.tolist() == [0, T, 2 * T] + [2 * T] * 6
     x_cpu = x.cpu()
