@@ -291,7 +291,7 @@ def test_pack_weight_is_a_transpose(m, tiny_handle):
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
     for which, shape in ((0, (8, 256, 512)), (1, (8, 512, 256))):
-        w = torch.randint(-127, 128, shape, generator=g, device="cuda", dtype=torch.int8)
+        w = torch.randint(-128, 128, shape, generator=g, device="cuda", dtype=torch.int8)
         p = torch.empty((shape[0], shape[2], shape[1]), dtype=torch.int8, device="cuda")
         m.check(m.moe_pack_weight(h, w, p, which))
         torch.cuda.synchronize()
@@ -302,6 +302,29 @@ def test_pack_weight_is_a_transpose(m, tiny_handle):
         m.check(m.moe_pack_weight_n(h, part, guard, which, 3))
         torch.cuda.synchronize()
         assert torch.equal(guard[:3], part.transpose(1, 2)) and bool((guard[3] == 7).all())
+
+
+@pytest.mark.parametrize("T", [8, 300])
+def test_every_weight_byte(m, tiny_handle, tiny_inputs, T):
+    """Weights taking each of the 256 int8 values equally often, -128 included (the synthetic
+    draws stop at -127): both layouts' converters turn every value into its exact bf16.  One value
+    converted wrongly moves the outputs by about a fifth of their spread, far above the
+    tolerance."""
+    h, _, layout = tiny_handle
+    g = torch.Generator().manual_seed(77)
+    layer_cpu = dict(tiny_inputs.layers[0])
+    for key in ("wl", "wv", "w1"):
+        shape = layer_cpu[key].shape
+        n = layer_cpu[key].numel()
+        vals = (torch.arange(n) % 256 - 128).to(torch.int8)
+        layer_cpu[key] = vals[torch.randperm(n, generator=g)].view(shape).contiguous()
+    dev = parity.to_dev(layer_cpu)
+    if layout == m.MOE_LAYOUT_PACKED:
+        dev = m.pack_layer(h, dev)
+    x_cpu = tiny_inputs.x[:T]
+    run = parity.Run(h, x_cpu.cuda(), dev)
+    near = parity.check_routing(run, oracle.route(x_cpu, layer_cpu["router_w"]), 8)
+    parity.check_output(run, layer_cpu, x_cpu, parity.sample_tokens(run, T, 64), near)
 
 
 def test_tiny_maximum_token_count(m, tiny_handle):
