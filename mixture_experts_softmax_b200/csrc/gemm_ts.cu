@@ -504,7 +504,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 epilogue_sync();
                 if (*last_flag) __threadfence();   // the other pieces' sums, visible after their tickets
             }
-            if (whole) {
+            if (whole && UP && kCols == 64) {
+                // the 128-route up-projection: this warp's 64 columns of H, packed as bf16 pairs in
+                // registers, so that the accumulator goes back to the MMA issuers before the stores
+                // (8-column loads keep the peak at 16 accumulator registers beside the 32 packed)
+                uint32_t hp[32];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    float x0[8], x1[8];
+                    __syncwarp();   // tcgen05.ld is warp-collective (.sync.aligned): converge first
+                    tmem_ld8(tl + c0 + 8 * k, x0);
+                    tmem_ld8(tl + BN + c0 + 8 * k, x1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __nv_bfloat162 v = __floats2bfloat162_rn(gelu_tanh(sc0 * x0[2 * i]) * (sc1 * x1[2 * i]),
+                                                                       gelu_tanh(sc0 * x0[2 * i + 1]) * (sc1 * x1[2 * i + 1]));
+                        hp[4 * k + i] = *reinterpret_cast<const uint32_t *>(&v);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty(b));
+                // the tile's real rows are its first nreal rows (the rest pad the expert's segment)
+                __nv_bfloat16 *hrow = a.h + static_cast<size_t>(row0 + c0) * a.M + f;
+                const int lim = nreal - c0;   // this warp's real columns
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    if (2 * j < lim) *hrow = __ushort_as_bfloat16(hp[j] & 0xFFFFu);
+                    hrow += a.M;
+                    if (2 * j + 1 < lim) *hrow = __ushort_as_bfloat16(hp[j] >> 16);
+                    hrow += a.M;
+                }
+            } else if (whole) {
 #pragma unroll 1
                 for (int c = c0; c < c1; c += 16) {
                     float x0[16], x1[16];
