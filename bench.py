@@ -434,9 +434,12 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
             out_host.copy_(hio, non_blocking=True)
         api = "moe_block_forward x%d with pinned host copies of the residual stream" % w.blocks
     else:
+        # successive calls overlap each input copy with the previous call's layer
+        moe.check(moe.moe_set_host_overlap(h.h, 1))
+
         def e2e_step():
             moe.check(moe.moe_forward_host(h.h, T, x_host, *moe.layer_args(layers[0]), out_host, stream))
-        api = "moe_forward_host"
+        api = "moe_forward_host (moe_set_host_overlap on)"
     for _ in range(max(1, W // 2)):
         e2e_step()
     barrier(world, dev)

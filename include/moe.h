@@ -165,6 +165,20 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
                              void *out_host, void *stream);
 
 /*
+ * Host overlap for moe_forward_host (on = 1; 0, the default, turns it off).  With
+ * it on, successive host-buffer forwards of this handle alternate between two
+ * device staging slots, and each call copies x_host in on a copy stream of the
+ * handle, so the copy overlaps the previous call's layer; the layer and the copy
+ * of the result into out_host stay on `stream`.  The input copy waits for its
+ * slot's previous call and, where x_host overlaps the host output of the call
+ * before, for that output (layers chained through host memory), but not for other
+ * work enqueued earlier on `stream`: x_host must hold its values when the call is
+ * made.  Results are identical with overlap on or off.  Costs a second pair of
+ * [T, d] staging buffers.  Returns MOE_EINVAL for a NULL handle or another value.
+ */
+MOE_API int moe_set_host_overlap(moe_handle h, int on);
+
+/*
  * One residual MoE block ("Transformer stack and language model head": pre/post
  * RMSNorm around the MoE, h += h_dense), in place on the residual stream:
  *   u = bf16( RMSNorm(h; g_pre) ),   h <- bf16( h + RMSNorm( MoE(u); g_post ) )

@@ -41,6 +41,7 @@ EXPORTS = (
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
     "moe_set_weight_layout", "moe_pack_weight", "moe_route_noalloc",
     "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_set_cta_pairs", "moe_pack_weight_n",
+    "moe_set_host_overlap",
 )
 
 
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "moe_ep_experts": (I, [P, I, I, P, P, P, P, P, P, P, P, P, P]),
         "moe_ep_combine": (I, [P, I, P, P, P]),
         "moe_set_cta_pairs": (I, [P, I]),
+        "moe_set_host_overlap": (I, [P, I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -211,6 +213,10 @@ MOE_PAIRS_ALL = 3          # CTA pairs also for small batches (32-route plans)
 def moe_set_cta_pairs(h, mode: int) -> int:
     """GEMMs on CTA pairs: one of the MOE_PAIRS_* modes (MOE_PAIRS_LARGE_DOWN by default)."""
     return _lib.moe_set_cta_pairs(h, int(mode))
+
+
+def moe_set_host_overlap(h, on: int) -> int:
+    return _lib.moe_set_host_overlap(h, int(on))
 
 
 def moe_set_weight_layout(h, layout: int) -> int:

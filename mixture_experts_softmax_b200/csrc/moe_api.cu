@@ -54,6 +54,18 @@ struct moe_ctx {
     // GEMMs' last-wave tickets (one per SM)
     int *err = nullptr;
     DevBuf b_part;     // fp32 [num_sms, 128, 256]: the GEMMs' last-wave partial sums
+    // host-buffer forwards with host overlap on (moe_set_host_overlap): two staging slots, each
+    // x [T, d] then out [T, d] bf16, used by alternate calls.  A call copies its input in on
+    // copy_in, so it can overlap the previous call's layer on the caller's stream.
+    bool host_overlap = false;
+    DevBuf b_host[2];
+    int host_slot = 0;
+    cudaStream_t copy_in = nullptr;
+    cudaEvent_t ev_in[2] = {nullptr, nullptr};     // slot k's input has landed
+    cudaEvent_t ev_done[2] = {nullptr, nullptr};   // slot k's last call has copied its output out
+    bool slot_used[2] = {false, false};
+    const char *slot_out[2] = {nullptr, nullptr};  // the host output range of slot k's last call
+    size_t slot_out_bytes[2] = {0, 0};
     int rows_cap = 0;       // rows the xp / h buffers hold
     int route_cap = 0;      // T the route buffer holds
     int map_gen = 0;        // bumps when b_xp / b_h move
@@ -176,6 +188,7 @@ RouteLayout route_layout(int T, int E)
 
 int sync_last(moe_ctx *h)
 {
+    if (h->copy_in && cudaStreamSynchronize(h->copy_in) != cudaSuccess) return MOE_ECUDA;
     if (!h->used) return MOE_OK;
     return cudaStreamSynchronize(h->last_stream) == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
@@ -762,8 +775,14 @@ MOE_API int moe_destroy(moe_handle h)
 {
     if (!h) return MOE_OK;
     sync_last(h);
-    for (DevBuf *b : {&h->b_route, &h->b_rperm, &h->b_xp, &h->b_h, &h->b_slots, &h->b_stage, &h->b_ep})
+    for (DevBuf *b : {&h->b_route, &h->b_rperm, &h->b_xp, &h->b_h, &h->b_slots, &h->b_stage, &h->b_ep, &h->b_host[0],
+                      &h->b_host[1]})
         if (b->ptr) cudaFree(b->ptr);
+    for (int k = 0; k < 2; ++k) {
+        if (h->ev_in[k]) cudaEventDestroy(h->ev_in[k]);
+        if (h->ev_done[k]) cudaEventDestroy(h->ev_done[k]);
+    }
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
     if (h->err) cudaFree(h->err);
     if (h->b_part.ptr) cudaFree(h->b_part.ptr);
     for (auto &p : h->pending) {
@@ -878,13 +897,54 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((rc = begin_call(h, T, s)) != MOE_OK) return rc;
     const size_t xb = static_cast<size_t>(T) * h->d * 2;
-    char *xs = static_cast<char *>(h->b_stage.ptr);
+    if (!h->host_overlap) {
+        char *xs = static_cast<char *>(h->b_stage.ptr);
+        char *os = xs + xb;
+        if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ECUDA;
+        if ((rc = run_layer(h, T, xs, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, os, nullptr, nullptr, nullptr, 0.f,
+                            s)) != MOE_OK)
+            return rc;
+        if (cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+        return MOE_OK;
+    }
+    // host overlap: slot k alternates between calls; the input copy runs on copy_in
+    if (!h->copy_in) {
+        if (cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking) != cudaSuccess) return MOE_ECUDA;
+        for (int j = 0; j < 2; ++j)
+            if (cudaEventCreateWithFlags(&h->ev_in[j], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&h->ev_done[j], cudaEventDisableTiming) != cudaSuccess)
+                return MOE_ECUDA;
+    }
+    const int k = h->host_slot, o = k ^ 1;
+    if ((rc = ensure(h, h->b_host[k], 2 * xb)) != MOE_OK) return rc;
+    char *xs = static_cast<char *>(h->b_host[k].ptr);
     char *os = xs + xb;
-    if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ECUDA;
+    // the copy in waits for the slot's previous call, and for the other slot's pending output
+    // when this input overlaps it (layers chained through host memory)
+    const char *xh = static_cast<const char *>(x_host);
+    const bool reads_pending = h->slot_used[o] && xh < h->slot_out[o] + h->slot_out_bytes[o] && h->slot_out[o] < xh + xb;
+    if (h->slot_used[k] && cudaStreamWaitEvent(h->copy_in, h->ev_done[k], 0) != cudaSuccess) return MOE_ECUDA;
+    if (reads_pending && cudaStreamWaitEvent(h->copy_in, h->ev_done[o], 0) != cudaSuccess) return MOE_ECUDA;
+    if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, h->copy_in) != cudaSuccess ||
+        cudaEventRecord(h->ev_in[k], h->copy_in) != cudaSuccess || cudaStreamWaitEvent(s, h->ev_in[k], 0) != cudaSuccess)
+        return MOE_ECUDA;
     if ((rc = run_layer(h, T, xs, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, os, nullptr, nullptr, nullptr, 0.f, s)) !=
         MOE_OK)
         return rc;
-    if (cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+    if (cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaEventRecord(h->ev_done[k], s) != cudaSuccess)
+        return MOE_ECUDA;
+    h->slot_used[k] = true;
+    h->slot_out[k] = static_cast<const char *>(out_host);
+    h->slot_out_bytes[k] = xb;
+    h->host_slot = o;
+    return MOE_OK;
+}
+
+MOE_API int moe_set_host_overlap(moe_handle h, int on)
+{
+    if (!h || (on != 0 && on != 1)) return MOE_EINVAL;
+    h->host_overlap = on != 0;
     return MOE_OK;
 }
 

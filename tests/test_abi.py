@@ -171,3 +171,15 @@ def test_cta_pairs_modes(m):
         assert m.moe_set_cta_pairs(None, 1) == m.MOE_EINVAL
     finally:
         m.moe_destroy(h)
+
+
+def test_host_overlap_switch(m):
+    rc, h = m.moe_create(256, 512, 8, 2)
+    assert rc == m.MOE_OK
+    try:
+        assert m.moe_set_host_overlap(h, 1) == m.MOE_OK
+        assert m.moe_set_host_overlap(h, 0) == m.MOE_OK
+        assert m.moe_set_host_overlap(h, 2) == m.MOE_EINVAL
+        assert m.moe_set_host_overlap(None, 1) == m.MOE_EINVAL
+    finally:
+        m.moe_destroy(h)

@@ -125,6 +125,39 @@ def test_forward_host_matches_device_path(m, tiny_inputs, tiny_handle, T):
     assert torch.equal(out_host, run.out_h)
 
 
+def test_host_overlap_matches_serial(m, tiny_inputs, tiny_handle):
+    """moe_set_host_overlap: calls alternating between two staging slots, input copies on the
+    handle's copy stream, give the serial path's results bit for bit.  The chain feeds each
+    call's host output to the next call as its input (the copy in must wait for it), changes
+    T on the way (the slots grow) and ends on a small batch (the staged input is copied into
+    the routed-rows buffer)."""
+    h, layer, _ = tiny_handle
+    m.check(m.moe_set_router_bias(h, None))
+    m.check(m.moe_set_padding_mask(h, None))
+    sizes = [100, 100, 300, 300, 8]
+    x0 = tiny_inputs.x[:300].clone().pin_memory()
+
+    def chain():
+        outs = [torch.empty((T, 256), dtype=torch.bfloat16).pin_memory() for T in sizes]
+        src = x0
+        for i, (T, out) in enumerate(zip(sizes, outs)):
+            m.check(m.moe_forward_host(h, T, src, *m.layer_args(layer), out))
+            nxt = sizes[i + 1] if i + 1 < len(sizes) else 0
+            src = out if 0 < nxt <= T else x0    # the next call reads this output where it fits
+        m.check(m.moe_sync_status(h))
+        return outs
+
+    serial = chain()
+    try:
+        m.check(m.moe_set_host_overlap(h, 1))
+        overlapped = chain()
+        again = chain()
+    finally:
+        m.check(m.moe_set_host_overlap(h, 0))
+    for a, b, c in zip(serial, overlapped, again):
+        assert torch.equal(a, b) and torch.equal(a, c)
+
+
 def test_kernel_times_reported(m, tiny_inputs, tiny_handle):
     h, layer, _ = tiny_handle
     x = tiny_inputs.x[:64].cuda()
