@@ -235,6 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the down-projection that follows may be scheduled onto SMs as this grid's CTAs leave them
+    if (UP && threadIdx.x == 0) griddep_launch_dependents();
     const uint32_t tmem_base = misc[0];
     const int total = prefix[a.E];
     const WorkList wl = a.part ? make_work_list(total, gridDim.x, a.ksteps) : WorkList{total, 0, total};
@@ -326,6 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == kWarpTmaB) {
         // ---- bf16 activation tiles [BN r x 128 k] (two 64-wide boxes) -> operand ring --
+        // The down-projection is launched to overlap the up-projection's last CTAs (its weight
+        // loads and conversions do not depend on them): its activations, H, are read only once
+        // the up-projection has completed.
+        if (!UP) griddep_wait();
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_last();
             uint32_t st = 0, ph = 0, issued = 0, par = 0;
@@ -443,6 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c1_full = BN >= 32 || hc == 0 ? c0 + kCols : c0;
         volatile uint32_t *last_flag = misc + 2;
         const EpiOut eo{a.rperm, a.gate, a.h, a.slots, a.M, a.T};
+        // the down-projection's slots, pieces and tickets: after the up-projection has completed
+        if (!UP) griddep_wait();
         auto epilogue_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
         int it = 0;
         PS_VAR(c_ewait);
@@ -683,8 +691,23 @@ cudaError_t launch_one_ts(const CUtensorMap &a0, const CUtensorMap &a1, const CU
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    gemm_ts_kernel<UP, BN><<<grid, kThreads, C::SMEM, s>>>(a0, a1, b, args);
-    return cudaGetLastError();
+    if (UP) {
+        gemm_ts_kernel<UP, BN><<<grid, kThreads, C::SMEM, s>>>(a0, a1, b, args);
+        return cudaGetLastError();
+    }
+    // the down-projection: programmatic stream serialization lets its CTAs start as the
+    // up-projection's leave their SMs (the kernel waits for the up-projection where it must)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_ts_kernel<UP, BN>, a0, a1, b, args);
 }
 
 }  // namespace
