@@ -52,6 +52,7 @@ __device__ __forceinline__ float4 slot_sum(const CombineArgs &a, int t, int c)
 template <int MAXS>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a)
 {
+    griddep_wait();   // launched to overlap the down-projection's end: its slots first
     const int per_row = a.d >> 2;
     const size_t n = static_cast<size_t>(a.T) * per_row;
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -72,6 +73,7 @@ template <int MAXS>
 __global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
 {
     __shared__ float red[8];
+    griddep_wait();   // launched to overlap the down-projection's end: its slots first
     const int t = blockIdx.x;
     if (__ldg(a.idx + 2 * t) < 0) return;   // a padding token: the residual row passes through unchanged
     float ss = 0.f;
@@ -104,22 +106,27 @@ __global__ void __launch_bounds__(256) combine_postnorm_kernel(CombineArgs a)
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s)
 {
     if (a.T <= 0) return cudaSuccess;
+    // programmatic stream serialization: the blocks may be scheduled while the down-projection
+    // ends; each waits for it before reading the slots
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
     // one split (large batches): the plain loop; several: all split loads in flight together
     if (a.h_io) {
-        if (a.splits == 1)
-            combine_postnorm_kernel<1><<<a.T, 256, 0, s>>>(a);
-        else
-            combine_postnorm_kernel<kMaxSplits><<<a.T, 256, 0, s>>>(a);
-    } else {
-        const size_t n = static_cast<size_t>(a.T) * (a.d >> 2);
-        const size_t want = (n + 255) / 256;
-        const int grid = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
-        if (a.splits == 1)
-            combine_kernel<1><<<grid, 256, 0, s>>>(a);
-        else
-            combine_kernel<kMaxSplits><<<grid, 256, 0, s>>>(a);
+        cfg.gridDim = dim3(a.T);
+        return a.splits == 1 ? cudaLaunchKernelEx(&cfg, combine_postnorm_kernel<1>, a)
+                             : cudaLaunchKernelEx(&cfg, combine_postnorm_kernel<kMaxSplits>, a);
     }
-    return cudaGetLastError();
+    const size_t n = static_cast<size_t>(a.T) * (a.d >> 2);
+    const size_t want = (n + 255) / 256;
+    cfg.gridDim = dim3(static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16));
+    return a.splits == 1 ? cudaLaunchKernelEx(&cfg, combine_kernel<1>, a)
+                         : cudaLaunchKernelEx(&cfg, combine_kernel<kMaxSplits>, a);
 }
 
 }  // namespace moe

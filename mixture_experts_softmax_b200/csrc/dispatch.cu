@@ -201,6 +201,9 @@ __global__ void __launch_bounds__(kRouteTokenThreads) route_small_kernel(RouteAr
     __shared__ bool s_last;
     __shared__ float s_logit[kFusedMaxT][kExperts];
     __shared__ int s_idx[2 * kFusedMaxT], s_slot[2 * kFusedMaxT];
+    // the up-projection, launched next with programmatic serialization, may set up on free SMs
+    // (it waits for this grid before it reads anything)
+    if (threadIdx.x == 0) griddep_launch_dependents();
     const int t = blockIdx.x / S, sl = blockIdx.x - t * S;
     if (!is_padding(ra, t)) {   // uniform over the block
         const int per = (ra.d >> 3) / S;

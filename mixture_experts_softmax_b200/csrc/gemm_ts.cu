@@ -177,6 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmB, const GemmArgs a)
 {
     using C = CfgTS<UP, BN>;
+    // launched to overlap the previous kernel's end: the up-projection reads the routing from its
+    // first instruction on, so all of it waits for that kernel (the down-projection waits later)
+    if (UP) griddep_wait();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -235,8 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // the down-projection that follows may be scheduled onto SMs as this grid's CTAs leave them
-    if (UP && threadIdx.x == 0) griddep_launch_dependents();
+    // the next kernel (the down-projection after the up-projection, the combine after the
+    // down-projection) may be scheduled onto SMs as this grid's CTAs leave them
+    if (threadIdx.x == 0) griddep_launch_dependents();
     const uint32_t tmem_base = misc[0];
     const int total = prefix[a.E];
     const WorkList wl = a.part ? make_work_list(total, gridDim.x, a.ksteps) : WorkList{total, 0, total};
@@ -691,12 +695,9 @@ cudaError_t launch_one_ts(const CUtensorMap &a0, const CUtensorMap &a1, const CU
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    if (UP) {
-        gemm_ts_kernel<UP, BN><<<grid, kThreads, C::SMEM, s>>>(a0, a1, b, args);
-        return cudaGetLastError();
-    }
-    // the down-projection: programmatic stream serialization lets its CTAs start as the
-    // up-projection's leave their SMs (the kernel waits for the up-projection where it must)
+    // programmatic stream serialization: the CTAs may start while the previous kernel ends (the
+    // kernel waits for it where it must); the down-projection's weight streaming overlaps the
+    // up-projection's last CTAs
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
