@@ -158,6 +158,36 @@ def test_host_overlap_matches_serial(m, tiny_inputs, tiny_handle):
         assert torch.equal(a, b) and torch.equal(a, c)
 
 
+def test_host_overlap_streams_and_pageable_memory(m, tiny_inputs, tiny_handle):
+    """Host overlap across a change of stream between calls (the handle waits for the previous
+    stream) and with pageable host buffers (the copies are then synchronous): the serial
+    path's results, bit for bit."""
+    h, layer, _ = tiny_handle
+    m.check(m.moe_set_router_bias(h, None))
+    m.check(m.moe_set_padding_mask(h, None))
+    T = 200
+    x_pinned = tiny_inputs.x[:T].clone().pin_memory()
+    x_pageable = tiny_inputs.x[:T].clone()
+    ref = torch.empty_like(x_pinned).pin_memory()
+    m.check(m.moe_forward_host(h, T, x_pinned, *m.layer_args(layer), ref))
+    m.check(m.moe_sync_status(h))
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    try:
+        m.check(m.moe_set_host_overlap(h, 1))
+        for i, (x, st) in enumerate(((x_pinned, s1), (x_pageable, s2), (x_pinned, s2), (x_pageable, s1))):
+            out = torch.empty_like(x_pinned).pin_memory() if i % 2 == 0 else torch.empty_like(x_pageable)
+            m.check(m.moe_forward_host(h, T, x, *m.layer_args(layer), out, st))
+            outs.append((out, st))
+        for out, st in outs:
+            st.synchronize()
+        m.check(m.moe_sync_status(h))
+    finally:
+        m.check(m.moe_set_host_overlap(h, 0))
+    for out, _ in outs:
+        assert torch.equal(out, ref)
+
+
 def test_kernel_times_reported(m, tiny_inputs, tiny_handle):
     h, layer, _ = tiny_handle
     x = tiny_inputs.x[:64].cuda()
