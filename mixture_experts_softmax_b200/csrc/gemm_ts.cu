@@ -624,14 +624,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + box * (kBKT / 2) + j0 * 8;
                 __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
-                // each pair of 16-byte chunks (32 reduction elements = 16 TMEM columns) is stored as
-                // soon as it is converted, so the TMEM writes spread over the conversion work
-                static_assert(C::CH % 2 == 0, "chunks go to TMEM in pairs");
+                // each group of four 16-byte chunks (64 reduction elements = 32 TMEM columns) is stored
+                // with one 32-column store as soon as it is converted, so the TMEM writes spread over
+                // the conversion work in few, wide instructions
+                static_assert(C::CH % 4 == 0, "chunks go to TMEM in fours");
 #pragma unroll
-                for (int c = 0; c < C::CH; c += 2) {
-                    uint32_t words[16];
+                for (int c = 0; c < C::CH; c += 4) {
+                    uint32_t words[32];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
+                    for (int h = 0; h < 4; ++h) {
                         const uint4 vv = v[c + h];
                         words[8 * h + 0] = i8x2_to_bf16x2(vv.x, 0x4140);
                         words[8 * h + 1] = i8x2_to_bf16x2(vv.x, 0x4342);
@@ -642,15 +643,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         words[8 * h + 6] = i8x2_to_bf16x2(vv.w, 0x4140);
                         words[8 * h + 7] = i8x2_to_bf16x2(vv.w, 0x4342);
                     }
-                    if (a.kblock) {   // dequantised weight bf16(w * s): exact w, one rounding of the product
+                    if (a.kblock) {
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
+                        for (int q = 0; q < 32; ++q) {
                             __nv_bfloat162 wq = *reinterpret_cast<const __nv_bfloat162 *>(&words[q]);
                             wq = __hmul2(wq, sc2);
                             words[q] = *reinterpret_cast<const uint32_t *>(&wq);
                         }
                     }
-                    tmem_st16(taddr + c * 8, words);
+                    tmem_st32(taddr + c * 8, words);
                 }
                 PS_ADD(c_cwork, t1);
                 PS_NOW(t2);
