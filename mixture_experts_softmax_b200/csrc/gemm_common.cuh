@@ -30,6 +30,21 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint
            (static_cast<uint64_t>(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor as its two 32-bit halves: the low word holds the address field and the
+// leading byte offset, the high word the stride, the version and the swizzle mode.  For a
+// 16-byte-aligned shared-memory address below 256 KB, moving the operand by off bytes (a multiple
+// of 16) adds off >> 4 to the low word and nothing else, so an MMA loop forms each descriptor
+// with one 32-bit add.
+__device__ __forceinline__ uint32_t desc_sw128_lo(uint32_t addr, uint32_t lbo)
+{
+    return ((addr & 0x3FFFFu) >> 4) | ((lbo >> 4) << 16);
+}
+__host__ __device__ constexpr uint32_t desc_sw128_hi(uint32_t sbo) { return (sbo >> 4) | (1u << 14) | (2u << 29); }
+__device__ __forceinline__ uint64_t desc_join(uint32_t lo, uint32_t hi)
+{
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Two signed bytes (chosen by `sel`) -> two exact bf16 values.  With the byte b in
 // the low 7 mantissa bits under exponent 2^7, hi = 128 + (b & 127); lo is 128, or
 // 256 when b's sign bit is set (it lands on the exponent's lowest bit); hi - lo = b

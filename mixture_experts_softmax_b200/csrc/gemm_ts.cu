@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     PS_NOW(t3);
                     tc_fence_after();
                     const uint32_t acol = tmem_base + C::A_BASE + st * C::A_COLS;
-                    const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
+                    const uint32_t blo = desc_sw128_lo(sbase + C::OFF_B + st * C::BBYTES, 16);
 #pragma unroll
                     for (int bx = 0; bx < C::NB; ++bx) {
 #pragma unroll
@@ -418,8 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // up-projection use the same slices, the k-boxes of the down-projection
                             // consecutive ones
                             const int kg = (UP ? 0 : bx * (kBKT / 16)) + kk;
-                            const uint64_t bdesc =
-                                desc_sw128(bbase + (kg >> 2) * (C::TN * 128) + (kg & 3) * 32, 16, 1024);
+                            const uint64_t bdesc = desc_join(
+                                blo + (((kg >> 2) * (C::TN * 128) + (kg & 3) * 32) >> 4), desc_sw128_hi(1024));
                             // the item's first MMA into an accumulator starts it
                             const int kr = ks - wi.k0;
                             const uint32_t acc = C::DUAL ? ((kr | kk) != 0) : ((kr | bx | kk) != 0);

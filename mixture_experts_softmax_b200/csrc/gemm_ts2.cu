@@ -411,14 +411,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     PS_NOW(t3);
                     tc_fence_after();
                     const uint32_t acol = tmem_base + C::A_BASE + st * C::A_COLS + mine * (kBKT / 2);
-                    const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
+                    const uint32_t blo = desc_sw128_lo(sbase + C::OFF_B + st * C::BBYTES, 16);
 #pragma unroll
                     for (int kk = 0; kk < kBKT / 16; ++kk) {
                         // K slice of the stage's activation tile: both matrices of the up-projection
                         // use the same slices, the k-boxes of the down-projection consecutive ones
                         const int kg = (UP ? 0 : mine * (kBKT / 16)) + kk;
-                        const uint64_t bdesc =
-                            desc_sw128(bbase + (kg >> 2) * (C::HALF * 128) + (kg & 3) * 32, 16, 1024);
+                        const uint64_t bdesc = desc_join(
+                            blo + (((kg >> 2) * (C::HALF * 128) + (kg & 3) * 32) >> 4), desc_sw128_hi(1024));
                         umma_bf16_ts_pair(dcol, acol + kk * 8, bdesc, idesc_pair<TN>(), ((ks - wi.k0) | kk) != 0);
                     }
                     issued_any = true;
