@@ -210,14 +210,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ks = 0; ks < a.ksteps; ++ks) {
                     if (!w.wait(a_full(st), ph, 4) || !w.wait(b_full(st), ph, 5)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t abase = sbase + C::OFF_A + st * C::ABYTES;
-                    const uint32_t bbase = sbase + C::OFF_B + st * C::BBYTES;
+                    // descriptor low words once per stage; each MMA adds its offset in 16-byte units
+                    const uint32_t alo = desc_sw128_lo(sbase + C::OFF_A + st * C::ABYTES, 1024);
+                    const uint32_t blo = desc_sw128_lo(sbase + C::OFF_B + st * C::BBYTES, 16);
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t bdesc = desc_sw128(bbase + kk * 32, 16, 1024);
+                        const uint64_t bdesc = desc_join(blo + ((kk * 32) >> 4), desc_sw128_hi(1024));
 #pragma unroll
                         for (int mat = 0; mat < C::NA; ++mat) {
-                            const uint64_t adesc = desc_sw128(abase + mat * kBM * kBK * 2 + kk * 4096, 1024, 2048);
+                            const uint64_t adesc =
+                                desc_join(alo + ((mat * kBM * kBK * 2 + kk * 4096) >> 4), desc_sw128_hi(2048));
                             umma_bf16(dcol + mat * BN, adesc, bdesc, idesc, (ks | kk) != 0);
                         }
                     }
