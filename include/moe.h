@@ -61,6 +61,8 @@ extern "C" {
 #define MOE_ECUDA        -4   /* a CUDA runtime call or kernel launch failed               */
 #define MOE_ETIMEOUT     -5   /* a bounded device-side wait ran out (see moe_sync_status)  */
 #define MOE_ENODEV       -6   /* no CUDA device, or not an sm_100 device                   */
+#define MOE_ERANGE       -7   /* a weight value the requested layout cannot hold (-128 in  */
+                              /* MOE_LAYOUT_PACKED; see moe_pack_weight)                   */
 
 /* Largest token count one call accepts. */
 #define MOE_MAX_TOKENS   262144
@@ -253,12 +255,18 @@ MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
  *   MOE_LAYOUT_IN_OUT (default)  [E, in, out]: the layout block above;
  *   MOE_LAYOUT_PACKED            [E, out, in]: each output feature's input
  *                                elements contiguous (w_lin, w_v [E, F, d];
- *                                w_1 [E, d, F]); written by moe_pack_weight.
+ *                                w_1 [E, d, F]), each value in sign-magnitude
+ *                                form; written by moe_pack_weight.
  * Both give the same result up to fp32 summation order.  With MOE_LAYOUT_PACKED
  * the GEMMs keep the dequantised bf16 weights in tensor memory instead of shared
- * memory: the fast path.  The layout change is a one-time cost at weight-load
- * time.  Scales are the same in both layouts.  Returns MOE_EINVAL for an
- * unknown layout.
+ * memory: the fast path.  There a weight w enters the tensor cores as the bf16
+ * w * 2^-133 (zero exponent field, |w| as the mantissa: two instructions per pair
+ * of weights), the routed rows and H at 2^64 times their values, and the
+ * epilogues take the products back by exact powers of two; so the packed path
+ * holds weights in [-127, 127] (symmetric int8 quantisation), scales below 2^59
+ * and routed rows and H (gelu(x W) * (x V)) below 2^64 in magnitude.  The layout change is a one-time cost at weight-load
+ * time.  Scales are the same in both layouts.  Returns MOE_EINVAL for an unknown
+ * layout.
  */
 MOE_API int moe_set_weight_layout(moe_handle h, int layout);
 
@@ -286,11 +294,14 @@ MOE_API int moe_set_weight_layout(moe_handle h, int layout);
 MOE_API int moe_set_cta_pairs(moe_handle h, int mode);
 
 /*
- * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT to MOE_LAYOUT_PACKED
- * (a per-expert transpose; values copied unchanged), enqueued on `stream`.
+ * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT to MOE_LAYOUT_PACKED: a
+ * per-expert transpose, each value w stored as the byte (w < 0 ? 0x80 : 0) | |w|.
  *   which = 0: w is linear or linear_v, [E, d, F] -> w_packed [E, F, d]
  *   which = 1: w is linear_1,           [E, F, d] -> w_packed [E, d, F]
- * w and w_packed are device buffers of E*d*F bytes that must not overlap.
+ * w and w_packed are device buffers of E*d*F bytes that must not overlap.  The
+ * call synchronises `stream` (a load-time step) and returns MOE_ERANGE if w holds
+ * -128, which has no packed form (w_packed is then not usable; such weights run
+ * in MOE_LAYOUT_IN_OUT, which holds every int8 value).
  */
 MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream);
 

@@ -26,6 +26,7 @@ MOE_ENOMEM = -3
 MOE_ECUDA = -4
 MOE_ETIMEOUT = -5
 MOE_ENODEV = -6
+MOE_ERANGE = -7
 MOE_MAX_TOKENS = 262144
 MOE_LAYOUT_IN_OUT = 0
 MOE_LAYOUT_PACKED = 1

@@ -109,8 +109,8 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
     dispatch_block<kDispatchThreads>(a);
 }
 
-// Xp[slot_of_route[2t + j], :] = x[t, :] for the T tokens and their two routes; 16-byte
-// copies, each token row read once.  Padding rows are left as they are: every MMA output
+// Xp[slot_of_route[2t + j], :] = x[t, :] (times kActScale when g.scaled) for the T tokens and
+// their two routes; 16-byte copies, each token row read once.  Padding rows are left as they are: every MMA output
 // column depends on its own B row only, and both GEMM epilogues skip rows whose route id
 // is -1.  The calling block takes groups of kGatherTokens tokens (group0, group0 + step,
 // ...), its threads the row's chunks, with the group's loads in flight together.
@@ -132,8 +132,9 @@ __device__ __forceinline__ void gather_rows(const GatherArgs &g, int T, const in
                 if (u < n) {   // slot -1: a padding token's route
                     const int r = 2 * (t0 + u);
                     const int p0 = slot_of_route[r], p1 = slot_of_route[r + 1];
-                    if (p0 >= 0) reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(p0) * g.d)[c] = v[u];
-                    if (p1 >= 0) reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(p1) * g.d)[c] = v[u];
+                    const uint4 o = g.scaled ? scale_bf16x8(v[u], kActScale) : v[u];
+                    if (p0 >= 0) reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(p0) * g.d)[c] = o;
+                    if (p1 >= 0) reinterpret_cast<uint4 *>(g.xp + static_cast<size_t>(p1) * g.d)[c] = o;
                 }
             }
         }

@@ -79,9 +79,9 @@ __global__ void __launch_bounds__(kLayoutThreads) ep_layout_kernel(EpLayoutArgs 
         for (int r = s_poff[k] + s_tot[k] + tid; r < s_poff[k + 1]; r += kLayoutThreads) a.rperm[r] = -1;
 }
 
-// xp[slot[i]] = rows[i] for the R received rows, 16-byte copies
+// xp[slot[i]] = rows[i] (times kActScale when `scaled`) for the R received rows, 16-byte copies
 __global__ void __launch_bounds__(256) ep_gather_kernel(int R, int d, const __nv_bfloat16 *rows, const int *slot,
-                                                       __nv_bfloat16 *xp)
+                                                       __nv_bfloat16 *xp, int scaled)
 {
     const int per_row = d >> 3;
     const size_t n = static_cast<size_t>(R) * per_row;
@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(256) ep_gather_kernel(int R, int d, const __nv
          q += static_cast<size_t>(gridDim.x) * blockDim.x) {
         const int i = static_cast<int>(q / per_row), c = static_cast<int>(q % per_row);
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(rows + static_cast<size_t>(i) * d) + c);
-        reinterpret_cast<uint4 *>(xp + static_cast<size_t>(__ldg(slot + i)) * d)[c] = v;
+        reinterpret_cast<uint4 *>(xp + static_cast<size_t>(__ldg(slot + i)) * d)[c] =
+            scaled ? scale_bf16x8(v, kActScale) : v;
     }
 }
 
@@ -154,11 +155,11 @@ cudaError_t launch_ep_layout(const EpLayoutArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-cudaError_t launch_ep_gather(int R, int d, const __nv_bfloat16 *rows, const int *slot, __nv_bfloat16 *xp,
+cudaError_t launch_ep_gather(int R, int d, const __nv_bfloat16 *rows, const int *slot, __nv_bfloat16 *xp, int scaled,
                              cudaStream_t s)
 {
     if (R <= 0) return cudaSuccess;
-    ep_gather_kernel<<<grid_for(static_cast<size_t>(R) * (d >> 3)), 256, 0, s>>>(R, d, rows, slot, xp);
+    ep_gather_kernel<<<grid_for(static_cast<size_t>(R) * (d >> 3)), 256, 0, s>>>(R, d, rows, slot, xp, scaled);
     return cudaGetLastError();
 }
 

@@ -45,7 +45,8 @@ __device__ __forceinline__ uint64_t desc_join(uint32_t lo, uint32_t hi)
     return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// Two signed bytes (chosen by `sel`) -> two exact bf16 values.  With the byte b in
+// Two signed bytes (chosen by `sel`) -> two exact bf16 values (the [E, in, out] layout's
+// weights, two's complement).  With the byte b in
 // the low 7 mantissa bits under exponent 2^7, hi = 128 + (b & 127); lo is 128, or
 // 256 when b's sign bit is set (it lands on the exponent's lowest bit); hi - lo = b
 // exactly (an integer of at most 8 significant bits).
@@ -57,6 +58,91 @@ __device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w, uint32_t sel)
     __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&hi),
                                *reinterpret_cast<const __nv_bfloat162 *>(&lo));
     return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// The packed (sign-magnitude) form of the same conversion.  prmt with a selector nibble of
+// 8 + i writes byte i's sign bit into all 8 bits of the result byte, so p holds, in each
+// 16-bit half, the sign replicated over the high byte above the packed byte itself.
+//   sm8x2_to_bf16x2_sub:   keep the sign bit and the 7 magnitude bits: the bf16 +-m * 2^-133
+//                          (zero exponent field), exactly w * 2^-133;
+//   sm8x2_to_bf16x2_exact: the normal bf16 w itself, as (+-(128 + m)) - (+-128): both terms
+//                          have exponent 2^7 and the sign of w, and their difference is exact.
+// `sel` picks bytes 0, 1 (0x9180) or bytes 2, 3 (0xB3A2) of the packed word.
+__device__ __forceinline__ uint32_t sm8x2_sign_spread(uint32_t w, uint32_t sel)
+{
+    uint32_t p;
+    asm("prmt.b32 %0, %1, %1, %2;" : "=r"(p) : "r"(w), "r"(sel));
+    return p;
+}
+__device__ __forceinline__ uint32_t sm8x2_to_bf16x2_sub(uint32_t w, uint32_t sel)
+{
+    return sm8x2_sign_spread(w, sel) & 0x807F807Fu;
+}
+__device__ __forceinline__ uint32_t sm8x2_to_bf16x2_exact(uint32_t w, uint32_t sel)
+{
+    const uint32_t p = sm8x2_sign_spread(w, sel);
+    const uint32_t hi = (p & 0x807F807Fu) | 0x43004300u;
+    const uint32_t lo = (p & 0x80008000u) | 0x43004300u;
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&hi),
+                               *reinterpret_cast<const __nv_bfloat162 *>(&lo));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+constexpr uint32_t kSelLo = 0x9180u, kSelHi = 0xB3A2u;
+
+// One 16-byte chunk of packed weights (16 values) -> 8 bf16 pairs for one 8-column TMEM store,
+// in the form convert_group describes.
+template <bool KBLOCK>
+__device__ __forceinline__ void convert_chunk(const uint4 &v, uint32_t (&words)[8], __nv_bfloat162 sc2)
+{
+    const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if constexpr (KBLOCK) {
+            words[2 * j] = sm8x2_to_bf16x2_exact(q[j], kSelLo);
+            words[2 * j + 1] = sm8x2_to_bf16x2_exact(q[j], kSelHi);
+        } else {
+            words[2 * j] = sm8x2_to_bf16x2_sub(q[j], kSelLo);
+            words[2 * j + 1] = sm8x2_to_bf16x2_sub(q[j], kSelHi);
+        }
+    }
+    if constexpr (KBLOCK) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            __nv_bfloat162 wq = *reinterpret_cast<const __nv_bfloat162 *>(&words[k]);
+            wq = __hmul2(wq, sc2);
+            words[k] = *reinterpret_cast<const uint32_t *>(&wq);
+        }
+    }
+}
+
+// Four 16-byte chunks of packed weights (64 values) -> 32 bf16 pairs for one 32-column TMEM
+// store: the subnormal form (per-channel scales, applied in the epilogue), or the exact
+// values times the block scale sc2 (per-block scales).
+template <bool KBLOCK>
+__device__ __forceinline__ void convert_group(const uint4 *v, uint32_t (&words)[32], __nv_bfloat162 sc2)
+{
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint32_t q[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if constexpr (KBLOCK) {
+                words[8 * h + 2 * j] = sm8x2_to_bf16x2_exact(q[j], kSelLo);
+                words[8 * h + 2 * j + 1] = sm8x2_to_bf16x2_exact(q[j], kSelHi);
+            } else {
+                words[8 * h + 2 * j] = sm8x2_to_bf16x2_sub(q[j], kSelLo);
+                words[8 * h + 2 * j + 1] = sm8x2_to_bf16x2_sub(q[j], kSelHi);
+            }
+        }
+    }
+    if constexpr (KBLOCK) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            __nv_bfloat162 wq = *reinterpret_cast<const __nv_bfloat162 *>(&words[k]);
+            wq = __hmul2(wq, sc2);
+            words[k] = *reinterpret_cast<const uint32_t *>(&wq);
+        }
+    }
 }
 
 __device__ __forceinline__ float gelu_tanh(float a)

@@ -99,8 +99,10 @@ __device__ __forceinline__ constexpr uint32_t idesc_ts()
 }
 
 // The tile epilogue on columns c .. c+15 of one accumulator row (TMEM lane = feature f),
-// from the full-K sums x0 (and x1: the second matrix, or the second k-box):
-//   up-projection:   H[r, f] = bf16( gelu(s0 * x0) * (s1 * x1) )
+// from the full-K sums x0 (and x1: the second matrix, or the second k-box).  The packed
+// operands are scaled (kActScale): sc0 and sc1 are the scales times the factor taking a sum
+// to its value.
+//   up-projection:   H[r, f] = bf16( gelu(s0 * x0) * (s1 * x1) ), stored at kActScale times it
 //   down-projection: slot[s, t, j, f] = gate[t, j] * s0 * (x0 + x1)   (k-box sums in this order)
 // padding rows (route id -1; for the up-projection: tile rows from nreal on) are skipped.
 struct EpiOut {
@@ -121,7 +123,8 @@ __device__ __forceinline__ void epilogue_chunk(const EpiOut &a, int row0, int nr
         for (int i = 0; i < 16; ++i) {
             const int r = row0 + c + i;
             if (c + i < nreal)
-                a.h[static_cast<size_t>(r) * a.M + f] = __float2bfloat16_rn(gelu_tanh(sc0 * x0[i]) * (sc1 * x1[i]));
+                a.h[static_cast<size_t>(r) * a.M + f] =
+                    __float2bfloat16_rn(gelu_tanh(sc0 * x0[i]) * (sc1 * x1[i]) * kActScale);
         }
     } else {
 #pragma unroll
@@ -168,6 +171,24 @@ __device__ __noinline__ void finish_pieces(const EpiOut a, const float *p0, int 
             }
         }
         epilogue_chunk<UP, NACC>(a, row0, nreal, c, f, s, sc0, sc1, x0, x1);
+    }
+}
+
+// One converter thread's share of a stage in the per-block scale format: CH 16-byte chunks of
+// its feature row (chunks j0 .. j0+CH-1, 128-byte swizzle: chunk j at (j ^ sw) * 16) loaded from
+// the staging ring at src, each value turned into bf16(w * scale), stored to TMEM at taddr.
+template <int CH>
+__device__ __noinline__ void convert_stage_kblock(uint32_t src, int j0, int sw, uint32_t taddr, __nv_bfloat162 sc2)
+{
+    uint4 v[CH];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) v[c] = lds128(src + (((j0 + c) ^ sw) << 4));
+    __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
+#pragma unroll
+    for (int c = 0; c < CH; c += 4) {
+        uint32_t words[32];
+        convert_group<true>(v + c, words, sc2);
+        tmem_st32(taddr + c * 8, words);
     }
 }
 
@@ -480,9 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nreal = roff[e + 1] - roff[e] - n * C::TN;   // real rows of this tile (may exceed TN)
             // a wide tile over an expert's odd last segment has BN columns
             const int c1 = C::WIDE ? max(c0, min(c1_full, poff[e + 1] - row0)) : c1_full;
-            // per-channel scales here; the per-block format applied them while dequantising
-            const float sc0 = a.kblock ? 1.f : __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
-            const float sc1 = !UP ? 0.f : a.kblock ? 1.f : __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
+            // per-channel scales here (the per-block format applied them while dequantising), times
+            // the factor taking a sum of scaled operands to its value: exact while |s| < 2^59
+            const float sc0 = (a.kblock ? 1.f : __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f])) * a.accf;
+            const float sc1 =
+                !UP ? 0.f : (a.kblock ? 1.f : __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f])) * a.accf;
             const bool whole = wi.piece < 0;   // uniform over the CTA
             if (!whole) {
                 // a piece: its partial sums go to the workspace, [piece][row][accumulator column]
@@ -530,8 +553,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const __nv_bfloat162 v = __floats2bfloat162_rn(gelu_tanh(sc0 * x0[2 * i]) * (sc1 * x1[2 * i]),
-                                                                       gelu_tanh(sc0 * x0[2 * i + 1]) * (sc1 * x1[2 * i + 1]));
+                        const float h0 = gelu_tanh(sc0 * x0[2 * i]) * (sc1 * x1[2 * i]);
+                        const float h1 = gelu_tanh(sc0 * x0[2 * i + 1]) * (sc1 * x1[2 * i + 1]);
+                        const __nv_bfloat162 v = __floats2bfloat162_rn(h0 * kActScale, h1 * kActScale);
                         hp[4 * k + i] = *reinterpret_cast<const uint32_t *>(&v);
                     }
                 }
@@ -614,44 +638,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 PS_NOW(t1);
                 tc_fence_after();
                 const uint32_t src = sbase + C::OFF_STG + st * C::STG + src_row;
-                uint4 v[C::CH];
-#pragma unroll
-                for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
-                __nv_bfloat162 sc2;   // this row's block scale (per-block format)
-                if (a.kblock) {
-                    const __nv_bfloat16 sv = srow[static_cast<size_t>(ks) * (C::KSTAGE / kScaleBlock) * a.M];
-                    sc2 = __halves2bfloat162(sv, sv);
-                }
                 const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + box * (kBKT / 2) + j0 * 8;
-                __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
-                // each group of four 16-byte chunks (64 reduction elements = 32 TMEM columns) is stored
-                // with one 32-column store as soon as it is converted, so the TMEM writes spread over
-                // the conversion work in few, wide instructions
                 static_assert(C::CH % 4 == 0, "chunks go to TMEM in fours");
+                if (a.kblock) {
+                    // this row's block scale (per-block format); out of line, so that this rarer
+                    // form does not add to the register pressure of the loop below
+                    const __nv_bfloat16 sv = srow[static_cast<size_t>(ks) * (C::KSTAGE / kScaleBlock) * a.M];
+                    convert_stage_kblock<C::CH>(src, j0, fr & 7, taddr, __halves2bfloat162(sv, sv));
+                } else {
+                    uint4 v[C::CH];
 #pragma unroll
-                for (int c = 0; c < C::CH; c += 4) {
-                    uint32_t words[32];
+                    for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
+                    __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
+                    // each group of four 16-byte chunks (64 reduction elements = 32 TMEM columns) is
+                    // stored with one 32-column store as soon as it is converted, so the TMEM writes
+                    // spread over the conversion work in few, wide instructions
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const uint4 vv = v[c + h];
-                        words[8 * h + 0] = i8x2_to_bf16x2(vv.x, 0x4140);
-                        words[8 * h + 1] = i8x2_to_bf16x2(vv.x, 0x4342);
-                        words[8 * h + 2] = i8x2_to_bf16x2(vv.y, 0x4140);
-                        words[8 * h + 3] = i8x2_to_bf16x2(vv.y, 0x4342);
-                        words[8 * h + 4] = i8x2_to_bf16x2(vv.z, 0x4140);
-                        words[8 * h + 5] = i8x2_to_bf16x2(vv.z, 0x4342);
-                        words[8 * h + 6] = i8x2_to_bf16x2(vv.w, 0x4140);
-                        words[8 * h + 7] = i8x2_to_bf16x2(vv.w, 0x4342);
+                    for (int c = 0; c < C::CH; c += 4) {
+                        uint32_t words[32];
+                        convert_group<false>(v + c, words, __nv_bfloat162{});
+                        tmem_st32(taddr + c * 8, words);
                     }
-                    if (a.kblock) {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) {
-                            __nv_bfloat162 wq = *reinterpret_cast<const __nv_bfloat162 *>(&words[q]);
-                            wq = __hmul2(wq, sc2);
-                            words[q] = *reinterpret_cast<const uint32_t *>(&wq);
-                        }
-                    }
-                    tmem_st32(taddr + c * 8, words);
                 }
                 PS_ADD(c_cwork, t1);
                 PS_NOW(t2);

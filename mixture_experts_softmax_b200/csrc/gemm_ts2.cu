@@ -144,8 +144,11 @@ __device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
-// The tile epilogue on columns c .. c+15 of this CTA's accumulator row (TMEM lane = feature f):
-//   up-projection:   H[r, f] = bf16( gelu(sc0 * x0) * (sc1 * x1) ) for the tile's real rows;
+// The tile epilogue on columns c .. c+15 of this CTA's accumulator row (TMEM lane = feature f).
+// The packed operands are scaled (kActScale): sc0 and sc1 are the scales times the factor
+// taking a sum to its value.
+//   up-projection:   H[r, f] = bf16( gelu(sc0 * x0) * (sc1 * x1) ) for the tile's real rows,
+//                    stored at kActScale times it;
 //   down-projection: slot[s, t, j, f] = gate[t, j] * sc0 * (x0 + x1)   (k-box sums in box order)
 template <bool UP, int NACC>
 __device__ __forceinline__ void pair_epilogue_chunk(const GemmArgs &a, int row0, int nreal, int c, int f, int s,
@@ -157,7 +160,7 @@ __device__ __forceinline__ void pair_epilogue_chunk(const GemmArgs &a, int row0,
         for (int i = 0; i < 16; ++i) {
             if (c + i < nreal)
                 a.h[static_cast<size_t>(row0 + c + i) * a.M + f] =
-                    __float2bfloat16_rn(gelu_tanh(sc0 * x0[i]) * (sc1 * x1[i]));
+                    __float2bfloat16_rn(gelu_tanh(sc0 * x0[i]) * (sc1 * x1[i]) * kActScale);
         }
     } else {
 #pragma unroll
@@ -201,6 +204,25 @@ __device__ __noinline__ void pair_finish_pieces(const GemmArgs a, const float *p
             }
         }
         pair_epilogue_chunk<UP, NACC>(a, row0, nreal, c, f, s, sc0, sc1, x0, x1);
+    }
+}
+
+// One converter thread's share of a stage in the per-block scale format: CH 16-byte chunks of
+// its feature row (chunks j0 .. j0+CH-1, 128-byte swizzle: chunk j at (j ^ sw) * 16) loaded from
+// the staging ring at src, each value turned into bf16(w * scale), stored to TMEM at taddr.
+template <int CH>
+__device__ __noinline__ void pair_convert_stage_kblock(uint32_t src, int j0, int sw, uint32_t taddr,
+                                                       __nv_bfloat162 sc2)
+{
+    uint4 v[CH];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) v[c] = lds128(src + (((j0 + c) ^ sw) << 4));
+    __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        uint32_t words[8];
+        convert_chunk<true>(v[c], words, sc2);
+        tmem_st8(taddr + c * 8, words);
     }
 }
 
@@ -470,8 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nreal = roff[e + 1] - roff[e] - n * C::TN;   // real rows of this tile (may exceed TN)
             // the tile's own rows: a 256-route tile over an expert's odd last segment fills 128 columns
             const int c1 = max(c0, min(c0 + TN / 2, poff[e + 1] - row0));
-            const float sc0 = a.kblock ? 1.f : __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f]);
-            const float sc1 = !UP ? 0.f : a.kblock ? 1.f : __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f]);
+            // the scales times the factor taking a sum of scaled operands to its value (exact while
+            // |s| < 2^59); the per-block format applied its scales while dequantising
+            const float sc0 = (a.kblock ? 1.f : __bfloat162float(a.s0[static_cast<size_t>(e) * a.M + f])) * a.accf;
+            const float sc1 =
+                !UP ? 0.f : (a.kblock ? 1.f : __bfloat162float(a.s1[static_cast<size_t>(e) * a.M + f])) * a.accf;
             const bool whole = wi.piece < 0;   // uniform over the pair
             if (!whole) {
                 // a piece: this CTA's partial sums go to the workspace, [piece][cta][row][column]
@@ -568,36 +593,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 PS_NOW(t1);
                 tc_fence_after();
                 const uint32_t src = sbase + C::OFF_STG + st * C::STG + src_row;
-                uint4 v[C::CH];
-#pragma unroll
-                for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
-                __nv_bfloat162 sc2;
-                if (a.kblock) {
-                    const __nv_bfloat16 sv = srow[static_cast<size_t>(ks) * (C::KSTAGE / kScaleBlock) * a.M];
-                    sc2 = __halves2bfloat162(sv, sv);
-                }
                 const uint32_t taddr = tmem_base + lane_base + C::A_BASE + st2 * C::A_COLS + box * (kBKT / 2) + j0 * 8;
-                __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
+                if (a.kblock) {
+                    // per-block scale format, out of line (keeps the register pressure of the loop below)
+                    const __nv_bfloat16 sv = srow[static_cast<size_t>(ks) * (C::KSTAGE / kScaleBlock) * a.M];
+                    pair_convert_stage_kblock<C::CH>(src, j0, fr & 7, taddr, __halves2bfloat162(sv, sv));
+                } else {
+                    uint4 v[C::CH];
 #pragma unroll
-                for (int c = 0; c < C::CH; ++c) {
-                    uint32_t words[8];
-                    words[0] = i8x2_to_bf16x2(v[c].x, 0x4140);
-                    words[1] = i8x2_to_bf16x2(v[c].x, 0x4342);
-                    words[2] = i8x2_to_bf16x2(v[c].y, 0x4140);
-                    words[3] = i8x2_to_bf16x2(v[c].y, 0x4342);
-                    words[4] = i8x2_to_bf16x2(v[c].z, 0x4140);
-                    words[5] = i8x2_to_bf16x2(v[c].z, 0x4342);
-                    words[6] = i8x2_to_bf16x2(v[c].w, 0x4140);
-                    words[7] = i8x2_to_bf16x2(v[c].w, 0x4342);
-                    if (a.kblock) {
+                    for (int c = 0; c < C::CH; ++c) v[c] = lds128(src + (((j0 + c) ^ (fr & 7)) << 4));
+                    __syncwarp();   // tcgen05.st is warp-collective (.sync.aligned): converge first
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            __nv_bfloat162 wq = *reinterpret_cast<const __nv_bfloat162 *>(&words[k]);
-                            wq = __hmul2(wq, sc2);
-                            words[k] = *reinterpret_cast<const uint32_t *>(&wq);
-                        }
+                    for (int c = 0; c < C::CH; ++c) {
+                        uint32_t words[8];
+                        convert_chunk<false>(v[c], words, __nv_bfloat162{});
+                        tmem_st8(taddr + c * 8, words);
                     }
-                    tmem_st8(taddr + c * 8, words);
                 }
                 PS_ADD(c_cwork, t1);
                 PS_NOW(t2);

@@ -15,6 +15,34 @@ constexpr int kBM = 128;          // output features per GEMM tile (TMEM lanes)
 constexpr int kBK = 64;           // reduction elements per pipeline stage (128 B of bf16)
 constexpr int kMaxSplits = 8;     // K-splits of the down-projection
 
+// The packed weight layout and its operand scaling (the TMEM-operand GEMMs).  Packed weights
+// hold each int8 value w in sign-magnitude form: bit 7 the sign, bits 0..6 |w| (so w = -128 has
+// no packed form).  A converter turns the byte into the bf16 with that sign, a zero exponent
+// field and |w| as its mantissa: the value w * 2^-133, exactly (bf16 numbers with a zero
+// exponent field are the multiples of 2^-133 below 2^-126).  Products with such an operand are
+// 2^133 times too small, so the other operand, the routed rows and H, is kept at kActScale times
+// its value, which holds the fp32 accumulator above its own subnormal range for activations down
+// to about 1e-20; the epilogues multiply the scales by kAccScaleChannel.  Every step is an exact
+// power-of-two scaling, as long as the routed rows and H stay below 2^64 in magnitude (beyond
+// that their scaled copies overflow) and the scales below 2^59.  With per-block scales the converters form bf16(w * s) as
+// normal numbers instead, and the epilogues multiply by kActUnscale.
+constexpr float kActScale = 0x1p64f;
+constexpr float kActUnscale = 0x1p-64f;
+constexpr float kAccScaleChannel = 0x1p69f;   // 2^133 / kActScale
+
+// two bf16 values (a 32-bit pair) or eight (16 bytes) times f, through fp32: exact for a
+// power of two f while the results stay finite (bf16 subnormals are fp32 subnormals, kept
+// without flushing)
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t w, float f)
+{
+    const __nv_bfloat162 r = __floats2bfloat162_rn(__uint_as_float(w << 16) * f, __uint_as_float(w & 0xffff0000u) * f);
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float f)
+{
+    return make_uint4(scale_bf16x2(v.x, f), scale_bf16x2(v.y, f), scale_bf16x2(v.z, f), scale_bf16x2(v.w, f));
+}
+
 // device error word values (the first error wins)
 constexpr int kErrTimeoutBase = 0x1000;   // + wait site
 
@@ -31,6 +59,8 @@ struct RouteArgs {
     float eps;
     __nv_bfloat16 *u;           // [T, d]
     const uint8_t *mask;        // [T] padding mask (0 = padding: experts -1, gates 0) or nullptr
+    int u_scaled;               // 1: u is written at kActScale times its value (the small-batch
+                                //    routing launch, when u is the packed up-projection's operand)
 };
 
 struct DispatchArgs {
@@ -48,6 +78,7 @@ struct GatherArgs {
     int d;
     const __nv_bfloat16 *x;     // [T, d]
     __nv_bfloat16 *xp;          // [rows, d]; only the rows of real routes are written
+    int scaled;                 // 1: rows written at kActScale times their value (packed layout)
 };
 
 // one grouped GEMM of the layer:  for every expert e and padded row r of e
@@ -83,6 +114,9 @@ struct GemmArgs {
     // rows [T, K] with one-row boxes and each tile row is loaded from row rperm >> 1 of it
     // (no gathered copy); 0 = the B map covers the gathered rows [rows, K]
     int gather;
+    // TMEM-operand kernels (packed layout): the factor taking an accumulator to its value
+    // (kAccScaleChannel, or kActUnscale with per-block scales); H is written at kActScale
+    float accf;
 };
 
 struct CombineArgs {
@@ -121,7 +155,7 @@ struct EpCombineArgs {
 
 cudaError_t launch_ep_layout(const EpLayoutArgs &a, cudaStream_t s);
 // xp[slot[i]] = rows[i], i < R
-cudaError_t launch_ep_gather(int R, int d, const __nv_bfloat16 *rows, const int *slot, __nv_bfloat16 *xp,
+cudaError_t launch_ep_gather(int R, int d, const __nv_bfloat16 *rows, const int *slot, __nv_bfloat16 *xp, int scaled,
                              cudaStream_t s);
 // y[i] = sum_s part[s * plane + i * d ...], s ascending
 cudaError_t launch_ep_split_sum(int R, int d, int splits, size_t plane, const float *part, float *y, cudaStream_t s);
@@ -163,7 +197,8 @@ cudaError_t launch_gemm_down_pair(int bn, const CUtensorMap &w1, const CUtensorM
 // reduction elements per pipeline stage of the TMEM-operand GEMM (up- or down-projection, tile width bn)
 int gemm_ts_kstage(bool up, int bn);
 // out[e, m, k] = in[e, k, m] for E int8 [K, M] matrices (K, M multiples of 64)
-cudaError_t launch_transpose_i8(const int8_t *in, int8_t *out, int E, int K, int M, cudaStream_t s);
+cudaError_t launch_pack_i8(const int8_t *in, int8_t *out, int E, int K, int M, int *range_flag, cudaStream_t s);
+cudaError_t launch_scale_rows(const __nv_bfloat16 *in, __nv_bfloat16 *out, size_t n, float f, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 
 // dynamic shared memory each GEMM variant needs (for cudaFuncSetAttribute)

@@ -71,6 +71,7 @@ struct moe_ctx {
     int map_gen = 0;        // bumps when b_xp / b_h move
     int last_T = -1;
     int last_block_T = -1;  // T of the last forward if it was moe_block_forward (u is staged), else -1
+    bool stage_scaled = false;   // that staged u is at kActScale (packed small-batch path)
     int ep_T = -1;          // T of the last moe_ep_dispatch (its routing waits for moe_ep_combine), else -1
     DevBuf b_ep;            // expert-parallel layout of received rows: counts, offsets, poff, rperm, slot, ones
 
@@ -101,9 +102,18 @@ namespace {
 
 constexpr int kCtlWords = 1024;     // words of the handle's zeroed control block
 constexpr int kCtlRouteTicket = 32;
+constexpr int kCtlPackRange = 48;   // moe_pack_weight: set when a weight is -128
 constexpr int kCtlTickets = 64;     // first GEMM ticket
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// the GEMM epilogues' factor from an accumulator to its value: the packed layout's operands are
+// scaled (kActScale); the shared-memory kernels of the [E, in, out] layout ignore it
+float acc_factor(const moe_ctx *h)
+{
+    if (h->layout != MOE_LAYOUT_PACKED) return 1.f;
+    return h->kblock ? kActUnscale : kAccScaleChannel;
+}
 
 // the up- (up = true) or down-projection of plans of tile width bn on CTA pairs on this handle
 bool pairs_for(const moe_ctx *h, int bn, bool up)
@@ -468,14 +478,16 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     }
     DispatchArgs da{T, h->E, bn, idx, rw + L.counts, rw + L.offsets, poff, rw + L.perm, rperm, rw + L.slot};
     GatherArgs ga{h->d, g_pre ? u : routed, static_cast<__nv_bfloat16 *>(h->b_xp.ptr)};
+    ga.scaled = ts ? 1 : 0;   // the packed GEMMs take their B rows at kActScale
     // small batches on the TMEM-operand kernels: the routing launch leaves the routed rows in
-    // the staging buffer (copied there unless they already are) and the up-projection loads
-    // its B rows from it, so nothing is gathered
+    // the staging buffer at kActScale (in place when they were staged there) and the
+    // up-projection loads its B rows from it, so nothing is gathered
     const bool gather_in_gemm = small && ts;
     const CUtensorMap *m_b = m_xp;
     if (gather_in_gemm) {
         if ((rc = stage_map(h, &m_b)) != MOE_OK) return rc;
-        if (!g_pre && routed != u) ra.u = u;
+        ra.u = u;
+        ra.u_scaled = 1;
         ga.xp = nullptr;
     }
     if (small) {
@@ -511,6 +523,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
     up.timeout_ns = h->timeout_ns;
     up.kblock = h->kblock;
     up.gather = gather_in_gemm ? 1 : 0;
+    up.accf = acc_factor(h);
     if (ts) {
         up.part = static_cast<float *>(h->b_part.ptr);
         up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
@@ -532,6 +545,7 @@ int run_layer(moe_ctx *h, int T, const void *x, const float *router_w, const int
         return MOE_ECUDA;
 
     h->last_block_T = g_pre ? T : -1;
+    h->stage_scaled = g_pre && gather_in_gemm;   // u in the staging buffer is at kActScale
     h->ep_T = -1;   // the route buffer now holds this forward's routing
     CombineArgs ca{T, h->d, splits, static_cast<const float *>(h->b_slots.ptr), idx, static_cast<__nv_bfloat16 *>(out),
                    static_cast<__nv_bfloat16 *>(h_io), static_cast<const __nv_bfloat16 *>(g_post), eps};
@@ -686,7 +700,7 @@ int run_ep_experts(moe_ctx *h, int n_src, int E_local, const int32_t *counts, in
     if (timed(h, K_DISPATCH, s, [&] { return launch_ep_layout(la, s); }) != cudaSuccess) return MOE_ECUDA;
     if (timed(h, K_GATHER, s, [&] {
             return launch_ep_gather(R, h->d, static_cast<const __nv_bfloat16 *>(recv_rows), la.slot,
-                                    static_cast<__nv_bfloat16 *>(h->b_xp.ptr), s);
+                                    static_cast<__nv_bfloat16 *>(h->b_xp.ptr), ts ? 1 : 0, s);
         }) != cudaSuccess)
         return MOE_ECUDA;
 
@@ -708,6 +722,7 @@ int run_ep_experts(moe_ctx *h, int n_src, int E_local, const int32_t *counts, in
     up.timeout_ns = h->timeout_ns;
     up.kblock = h->kblock;
     up.gather = 0;
+    up.accf = acc_factor(h);
     if (ts) {
         up.part = static_cast<float *>(h->b_part.ptr);
         up.tickets = reinterpret_cast<unsigned int *>(h->err + kCtlTickets);
@@ -748,6 +763,7 @@ MOE_API const char *moe_strerror(int code)
     case MOE_ECUDA: return "CUDA error";
     case MOE_ETIMEOUT: return "device-side wait timed out";
     case MOE_ENODEV: return "no sm_100 CUDA device";
+    case MOE_ERANGE: return "weight value outside the layout's range";
     default: return "unknown status code";
     }
 }
@@ -850,9 +866,15 @@ MOE_API int moe_pack_weight_n(moe_handle h, const int8_t *w, int8_t *w_packed, i
     int rc = ensure_device(h);
     if (rc != MOE_OK) return rc;
     const int K = which == 0 ? h->d : h->F, M = which == 0 ? h->F : h->d;
-    return launch_transpose_i8(w, w_packed, n_experts, K, M, static_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? MOE_OK
-               : MOE_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int *flag = h->err + kCtlPackRange;
+    int minus128 = 0;
+    if (cudaMemsetAsync(flag, 0, sizeof(int), s) != cudaSuccess ||
+        launch_pack_i8(w, w_packed, n_experts, K, M, flag, s) != cudaSuccess ||
+        cudaMemcpyAsync(&minus128, flag, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return MOE_ECUDA;
+    return minus128 ? MOE_ERANGE : MOE_OK;
 }
 
 MOE_API int moe_pack_weight(moe_handle h, const int8_t *w, int8_t *w_packed, int which, void *stream)
@@ -987,11 +1009,14 @@ MOE_API int moe_get_routing(moe_handle h, int32_t *idx, float *gate, int32_t *of
 MOE_API int moe_get_block_input(moe_handle h, void *u, void *stream)
 {
     if (!h || !u || !aligned16(u) || h->last_block_T < 0) return MOE_EINVAL;
-    const size_t bytes = static_cast<size_t>(h->last_block_T) * h->d * 2;
-    return cudaMemcpyAsync(u, h->b_stage.ptr, bytes, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)) ==
-                   cudaSuccess
-               ? MOE_OK
-               : MOE_ECUDA;
+    const size_t n = static_cast<size_t>(h->last_block_T) * h->d;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        h->stage_scaled
+            ? launch_scale_rows(static_cast<const __nv_bfloat16 *>(h->b_stage.ptr), static_cast<__nv_bfloat16 *>(u), n,
+                                kActUnscale, s)
+            : cudaMemcpyAsync(u, h->b_stage.ptr, n * 2, cudaMemcpyDeviceToDevice, s);
+    return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 MOE_API int moe_sync_status(moe_handle h, void *stream)

@@ -1,15 +1,24 @@
 // pack.cu -- one-time weight layout change for the TMEM-operand GEMMs: every expert's
 // int8 matrix stored [in, out] (x @ W orientation) becomes [out, in], so that the
-// reduction elements of one output feature are contiguous.  Values are copied, not
-// changed; scales are untouched (they stay per output channel).
+// reduction elements of one output feature are contiguous, and each value w is stored in
+// sign-magnitude form (bit 7 the sign, bits 0..6 |w|), which the GEMMs' converters turn
+// into a bf16 operand in two instructions per pair of values (kActScale in kernels.cuh).
+// -128 has no such form: it is reported through `range_flag`.  Scales are untouched (they
+// stay per output channel).
 #include "kernels.cuh"
 
 namespace moe {
 
 namespace {
 
-// 64 x 64-byte tiles through shared memory: out[e, m, k] = in[e, k, m]
-__global__ void __launch_bounds__(256) transpose_i8_kernel(const int8_t *in, int8_t *out, int K, int M)
+// a two's-complement byte -> its sign-magnitude byte (-128 -> 0x80, flagged by the caller)
+__device__ __forceinline__ uint32_t sign_magnitude(uint32_t b)
+{
+    return (b & 0x80u) ? (0x80u | ((0x100u - b) & 0x7Fu)) : b;
+}
+
+// 64 x 64-byte tiles through shared memory: out[e, m, k] = sm(in[e, k, m])
+__global__ void __launch_bounds__(256) pack_i8_kernel(const int8_t *in, int8_t *out, int K, int M, int *range_flag)
 {
     __shared__ uint32_t tile[64][17];   // [k][m / 4], padded
     const int e = blockIdx.z, k0 = blockIdx.y * 64, m0 = blockIdx.x * 64;
@@ -22,26 +31,48 @@ __global__ void __launch_bounds__(256) transpose_i8_kernel(const int8_t *in, int
     __syncthreads();
     const int mm = threadIdx.x >> 2, ks = (threadIdx.x & 3) * 16;
     uint32_t w[4];
+    bool minus128 = false;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         uint32_t acc = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
             const uint32_t byte = (tile[ks + q * 4 + b][mm >> 2] >> (8 * (mm & 3))) & 0xffu;
-            acc |= byte << (8 * b);
+            minus128 |= byte == 0x80u;
+            acc |= sign_magnitude(byte) << (8 * b);
         }
         w[q] = acc;
     }
     *reinterpret_cast<uint4 *>(out + (static_cast<size_t>(e) * M + m0 + mm) * K + k0 + ks) =
         make_uint4(w[0], w[1], w[2], w[3]);
+    if (minus128) *range_flag = 1;
+}
+
+// out = in * f for n bf16 values (n a multiple of 8), in fp32: exact for a power of two f
+// while the results stay finite
+__global__ void __launch_bounds__(256) scale_rows_kernel(const uint4 *in, uint4 *out, size_t n8, float f)
+{
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        out[i] = scale_bf16x8(in[i], f);
 }
 
 }  // namespace
 
-cudaError_t launch_transpose_i8(const int8_t *in, int8_t *out, int E, int K, int M, cudaStream_t s)
+cudaError_t launch_pack_i8(const int8_t *in, int8_t *out, int E, int K, int M, int *range_flag, cudaStream_t s)
 {
     dim3 grid(M / 64, K / 64, E);
-    transpose_i8_kernel<<<grid, 256, 0, s>>>(in, out, K, M);
+    pack_i8_kernel<<<grid, 256, 0, s>>>(in, out, K, M, range_flag);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scale_rows(const __nv_bfloat16 *in, __nv_bfloat16 *out, size_t n, float f, cudaStream_t s)
+{
+    const size_t n8 = n / 8;
+    if (n8 == 0) return cudaSuccess;
+    const unsigned int blocks = static_cast<unsigned int>(n8 / 256 + 1 < 4096 ? n8 / 256 + 1 : 4096);
+    scale_rows_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4 *>(in), reinterpret_cast<uint4 *>(out), n8,
+                                             f);
     return cudaGetLastError();
 }
 

@@ -161,7 +161,9 @@ __device__ __forceinline__ void route_token(const RouteArgs &a, int t)
 // RMS-normalised u of the residual block: the sum of squares is taken over the whole row
 // (the same fixed order in every block that calls this for token t, so all of them get the
 // same scale), and the slice's chunks of u are formed, rounded to bf16, stored to a.u and
-// used.  Without a.g_pre and with a.u set, the slice's chunks of x are copied to a.u.
+// used.  Without a.g_pre and with a.u set, the slice's chunks of x are copied to a.u (in place
+// when a.u is a.x: each chunk is read and written by one thread).  With a.u_scaled the chunks
+// go to a.u at kActScale times their value; the routing itself uses the values.
 __device__ __forceinline__ void route_slice(const RouteArgs &a, int t, int c0, int c1, float (&acc)[kExperts])
 {
     constexpr int kWarps = kRouteTokenThreads / 32;
@@ -210,7 +212,7 @@ __device__ __forceinline__ void route_slice(const RouteArgs &a, int t, int c0, i
             }
             v = make_uint4(uv[0], uv[1], uv[2], uv[3]);
         }
-        if (ur) ur[c] = v;
+        if (ur) ur[c] = a.u_scaled ? scale_bf16x8(v, kActScale) : v;
         dot8(v, w4, c * 8, acc);
     }
 #pragma unroll

@@ -350,41 +350,78 @@ def test_cta_pairs_match_single_cta(m, tiny_inputs, tiny_handle, T, mode):
     parity.check_output(paired, tiny_inputs.layers[0], tiny_inputs.x[:T], range(T), near)
 
 
-def test_pack_weight_is_a_transpose(m, tiny_handle):
+def _sign_magnitude(w):
+    """The packed byte of each int8 value: bit 7 the sign, bits 0..6 the magnitude."""
+    wi = w.to(torch.int16)
+    return torch.where(wi < 0, 0x80 | (-wi), wi).to(torch.uint8)
+
+
+def test_pack_weight_layout(m, tiny_handle):
+    """moe_pack_weight transposes each expert and stores every value of [-127, 127] in
+    sign-magnitude form; a tensor holding -128 is refused with MOE_ERANGE."""
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
     for which, shape in ((0, (8, 256, 512)), (1, (8, 512, 256))):
-        w = torch.randint(-128, 128, shape, generator=g, device="cuda", dtype=torch.int8)
+        w = torch.randint(-127, 128, shape, generator=g, device="cuda", dtype=torch.int8)
         p = torch.empty((shape[0], shape[2], shape[1]), dtype=torch.int8, device="cuda")
         m.check(m.moe_pack_weight(h, w, p, which))
         torch.cuda.synchronize()
-        assert torch.equal(p, w.transpose(1, 2))
+        assert torch.equal(p.view(torch.uint8), _sign_magnitude(w.transpose(1, 2)))
         # a rank's share of the experts: exactly its bytes are read and written
         part = w[2:5].contiguous()
         guard = torch.full((4, shape[2], shape[1]), 7, dtype=torch.int8, device="cuda")
         m.check(m.moe_pack_weight_n(h, part, guard, which, 3))
         torch.cuda.synchronize()
-        assert torch.equal(guard[:3], part.transpose(1, 2)) and bool((guard[3] == 7).all())
+        assert torch.equal(guard[:3].view(torch.uint8), _sign_magnitude(part.transpose(1, 2)))
+        assert bool((guard[3] == 7).all())
+        # one -128 anywhere: no packed form
+        w.view(-1)[12345] = -128
+        assert m.moe_pack_weight(h, w, p, which) == m.MOE_ERANGE
+        # and the range flag does not outlive the call
+        w.view(-1)[12345] = -127
+        m.check(m.moe_pack_weight(h, w, p, which))
 
 
 @pytest.mark.parametrize("T", [8, 300])
 def test_every_weight_byte(m, tiny_handle, tiny_inputs, T):
-    """Weights taking each of the 256 int8 values equally often, -128 included (the synthetic
-    draws stop at -127): both layouts' converters turn every value into its exact bf16.  One value
-    converted wrongly moves the outputs by about a fifth of their spread, far above the
-    tolerance."""
+    """Weights taking every int8 value the layout holds equally often: all 256 in the [E, in, out]
+    layout, -128 included (the synthetic draws stop at -127), and the 255 values of [-127, 127] in
+    the packed layout (-128 has no packed form: test_pack_weight_layout).  Each layout's
+    converters turn every value into its exact bf16 operand.  One value converted wrongly moves
+    the outputs by about a fifth of their spread, far above the tolerance."""
     h, _, layout = tiny_handle
     g = torch.Generator().manual_seed(77)
     layer_cpu = dict(tiny_inputs.layers[0])
+    lo = -127 if layout == m.MOE_LAYOUT_PACKED else -128
     for key in ("wl", "wv", "w1"):
         shape = layer_cpu[key].shape
         n = layer_cpu[key].numel()
-        vals = (torch.arange(n) % 256 - 128).to(torch.int8)
+        vals = (torch.arange(n) % (128 - lo) + lo).to(torch.int8)
         layer_cpu[key] = vals[torch.randperm(n, generator=g)].view(shape).contiguous()
     dev = parity.to_dev(layer_cpu)
     if layout == m.MOE_LAYOUT_PACKED:
         dev = m.pack_layer(h, dev)
     x_cpu = tiny_inputs.x[:T]
+    run = parity.Run(h, x_cpu.cuda(), dev)
+    near = parity.check_routing(run, oracle.route(x_cpu, layer_cpu["router_w"]), 8)
+    parity.check_output(run, layer_cpu, x_cpu, parity.sample_tokens(run, T, 64), near)
+
+
+@pytest.mark.parametrize("e", [-24, 24])
+@pytest.mark.parametrize("T", [8, 300])
+def test_activation_scale(m, tiny_handle, tiny_inputs, T, e):
+    """Activations 2^e times the synthetic draws (router weight 2^-e times, so the routing is
+    the same): the packed path keeps its operands at fixed power-of-two scales, so tiny and large
+    activations keep their relative accuracy (H, about quadratic in x, spans 2^-50 .. 2^50 here).
+    Without the scaled B operands the down-projection's sums at e = -24 (about 2^-170 before the
+    epilogue's factor) would underflow to zero."""
+    h, _, layout = tiny_handle
+    layer_cpu = dict(tiny_inputs.layers[0])
+    layer_cpu["router_w"] = layer_cpu["router_w"] * 2.0 ** -e
+    x_cpu = (tiny_inputs.x[:T].float() * 2.0 ** e).to(torch.bfloat16)
+    dev = parity.to_dev(layer_cpu)
+    if layout == m.MOE_LAYOUT_PACKED:
+        dev = m.pack_layer(h, dev)
     run = parity.Run(h, x_cpu.cuda(), dev)
     near = parity.check_routing(run, oracle.route(x_cpu, layer_cpu["router_w"]), 8)
     parity.check_output(run, layer_cpu, x_cpu, parity.sample_tokens(run, T, 64), near)
