@@ -255,13 +255,14 @@ MOE_API int moe_get_kernel_times(moe_handle h, float *ms, int *launches, int n);
  *   MOE_LAYOUT_IN_OUT (default)  [E, in, out]: the layout block above;
  *   MOE_LAYOUT_PACKED            [E, out, in]: each output feature's input
  *                                elements contiguous (w_lin, w_v [E, F, d];
- *                                w_1 [E, d, F]), each value in sign-magnitude
- *                                form; written by moe_pack_weight.
+ *                                w_1 [E, d, F]), one byte per value, each value
+ *                                as a sign and a 7-bit magnitude (layout below);
+ *                                written by moe_pack_weight.
  * Both give the same result up to fp32 summation order.  With MOE_LAYOUT_PACKED
  * the GEMMs keep the dequantised bf16 weights in tensor memory instead of shared
  * memory: the fast path.  There a weight w enters the tensor cores as the bf16
- * w * 2^-133 (zero exponent field, |w| as the mantissa: two instructions per pair
- * of weights), the routed rows and H at 2^64 times their values, and the
+ * w * 2^-133 (zero exponent field, |w| as the mantissa: three instructions per four
+ * weights), the routed rows and H at 2^64 times their values, and the
  * epilogues take the products back by exact powers of two; so the packed path
  * holds weights in [-127, 127] (symmetric int8 quantisation), scales below 2^59
  * and routed rows and H (gelu(x W) * (x V)) below 2^64 in magnitude.  The layout change is a one-time cost at weight-load
@@ -295,7 +296,9 @@ MOE_API int moe_set_cta_pairs(moe_handle h, int mode);
 
 /*
  * Rewrite one int8 weight tensor from MOE_LAYOUT_IN_OUT to MOE_LAYOUT_PACKED: a
- * per-expert transpose, each value w stored as the byte (w < 0 ? 0x80 : 0) | |w|.
+ * per-expert transpose; every four consecutive input elements w0..w3 of an output
+ * feature become the bytes  s2|m0, s0|m2, s3|m1, s1|m3  (mi = |wi|, si = 0x80 if wi < 0),
+ * the signs crossed over so that a mask, and a byte swap and a mask, give bf16 pairs.
  *   which = 0: w is linear or linear_v, [E, d, F] -> w_packed [E, F, d]
  *   which = 1: w is linear_1,           [E, F, d] -> w_packed [E, d, F]
  * w and w_packed are device buffers of E*d*F bytes that must not overlap.  The

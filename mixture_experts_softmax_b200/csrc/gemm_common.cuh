@@ -60,34 +60,34 @@ __device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w, uint32_t sel)
     return *reinterpret_cast<uint32_t *>(&r);
 }
 
-// The packed (sign-magnitude) form of the same conversion.  prmt with a selector nibble of
-// 8 + i writes byte i's sign bit into all 8 bits of the result byte, so p holds, in each
-// 16-bit half, the sign replicated over the high byte above the packed byte itself.
-//   sm8x2_to_bf16x2_sub:   keep the sign bit and the 7 magnitude bits: the bf16 +-m * 2^-133
-//                          (zero exponent field), exactly w * 2^-133;
-//   sm8x2_to_bf16x2_exact: the normal bf16 w itself, as (+-(128 + m)) - (+-128): both terms
-//                          have exponent 2^7 and the sign of w, and their difference is exact.
-// `sel` picks bytes 0, 1 (0x9180) or bytes 2, 3 (0xB3A2) of the packed word.
-__device__ __forceinline__ uint32_t sm8x2_sign_spread(uint32_t w, uint32_t sel)
+// The packed form.  A packed 32-bit word holds the weights of four consecutive reduction
+// elements k .. k+3, each as a sign bit and a 7-bit magnitude, with the signs crossed over within
+// each 16-bit half: byte 0 = sign(w[k+2]) << 7 | |w[k]|,   byte 1 = sign(w[k]) << 7 | |w[k+2]|,
+//                   byte 2 = sign(w[k+3]) << 7 | |w[k+1]|, byte 3 = sign(w[k+1]) << 7 | |w[k+3]|.
+// Masked with 0x807F807F the word is the bf16 pair (w[k], w[k+1]) with zero exponent fields:
+// the values w * 2^-133, exactly (bf16 numbers with a zero exponent field are the multiples of
+// 2^-133 below 2^-126).  With the bytes of each half swapped first (prmt 0x2301), the same mask
+// gives (w[k+2], w[k+3]).  Three integer instructions per two pairs.
+//   pk_lo / pk_hi:        the pairs (w[k], w[k+1]) / (w[k+2], w[k+3]) as w * 2^-133;
+//   pk_exact:             a masked-ready word's pair as the normal bf16 values w themselves, formed as
+//                         (+-(128 + m)) - (+-128): both terms have exponent 2^7 and the sign of w, and
+//                         their difference is exact.
+__device__ __forceinline__ uint32_t pk_swap(uint32_t q)
 {
     uint32_t p;
-    asm("prmt.b32 %0, %1, %1, %2;" : "=r"(p) : "r"(w), "r"(sel));
+    asm("prmt.b32 %0, %1, %1, 0x2301;" : "=r"(p) : "r"(q));
     return p;
 }
-__device__ __forceinline__ uint32_t sm8x2_to_bf16x2_sub(uint32_t w, uint32_t sel)
+__device__ __forceinline__ uint32_t pk_lo(uint32_t q) { return q & 0x807F807Fu; }
+__device__ __forceinline__ uint32_t pk_hi(uint32_t q) { return pk_swap(q) & 0x807F807Fu; }
+__device__ __forceinline__ uint32_t pk_exact(uint32_t q)
 {
-    return sm8x2_sign_spread(w, sel) & 0x807F807Fu;
-}
-__device__ __forceinline__ uint32_t sm8x2_to_bf16x2_exact(uint32_t w, uint32_t sel)
-{
-    const uint32_t p = sm8x2_sign_spread(w, sel);
-    const uint32_t hi = (p & 0x807F807Fu) | 0x43004300u;
-    const uint32_t lo = (p & 0x80008000u) | 0x43004300u;
+    const uint32_t hi = (q & 0x807F807Fu) | 0x43004300u;
+    const uint32_t lo = (q & 0x80008000u) | 0x43004300u;
     __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&hi),
                                *reinterpret_cast<const __nv_bfloat162 *>(&lo));
     return *reinterpret_cast<uint32_t *>(&r);
 }
-constexpr uint32_t kSelLo = 0x9180u, kSelHi = 0xB3A2u;
 
 // One 16-byte chunk of packed weights (16 values) -> 8 bf16 pairs for one 8-column TMEM store,
 // in the form convert_group describes.
@@ -98,11 +98,11 @@ __device__ __forceinline__ void convert_chunk(const uint4 &v, uint32_t (&words)[
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         if constexpr (KBLOCK) {
-            words[2 * j] = sm8x2_to_bf16x2_exact(q[j], kSelLo);
-            words[2 * j + 1] = sm8x2_to_bf16x2_exact(q[j], kSelHi);
+            words[2 * j] = pk_exact(q[j]);
+            words[2 * j + 1] = pk_exact(pk_swap(q[j]));
         } else {
-            words[2 * j] = sm8x2_to_bf16x2_sub(q[j], kSelLo);
-            words[2 * j + 1] = sm8x2_to_bf16x2_sub(q[j], kSelHi);
+            words[2 * j] = pk_lo(q[j]);
+            words[2 * j + 1] = pk_hi(q[j]);
         }
     }
     if constexpr (KBLOCK) {
@@ -127,11 +127,11 @@ __device__ __forceinline__ void convert_group(const uint4 *v, uint32_t (&words)[
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             if constexpr (KBLOCK) {
-                words[8 * h + 2 * j] = sm8x2_to_bf16x2_exact(q[j], kSelLo);
-                words[8 * h + 2 * j + 1] = sm8x2_to_bf16x2_exact(q[j], kSelHi);
+                words[8 * h + 2 * j] = pk_exact(q[j]);
+                words[8 * h + 2 * j + 1] = pk_exact(pk_swap(q[j]));
             } else {
-                words[8 * h + 2 * j] = sm8x2_to_bf16x2_sub(q[j], kSelLo);
-                words[8 * h + 2 * j + 1] = sm8x2_to_bf16x2_sub(q[j], kSelHi);
+                words[8 * h + 2 * j] = pk_lo(q[j]);
+                words[8 * h + 2 * j + 1] = pk_hi(q[j]);
             }
         }
     }

@@ -16,10 +16,11 @@ constexpr int kBK = 64;           // reduction elements per pipeline stage (128 
 constexpr int kMaxSplits = 8;     // K-splits of the down-projection
 
 // The packed weight layout and its operand scaling (the TMEM-operand GEMMs).  Packed weights
-// hold each int8 value w in sign-magnitude form: bit 7 the sign, bits 0..6 |w| (so w = -128 has
-// no packed form).  A converter turns the byte into the bf16 with that sign, a zero exponent
-// field and |w| as its mantissa: the value w * 2^-133, exactly (bf16 numbers with a zero
-// exponent field are the multiples of 2^-133 below 2^-126).  Products with such an operand are
+// hold each int8 value w as a sign bit and a 7-bit magnitude (so w = -128 has no packed form),
+// four consecutive reduction elements to a 32-bit word with the signs crossed over within each
+// 16-bit half (gemm_common.cuh, pk_lo).  A converter turns a value into the bf16 with its sign,
+// a zero exponent field and |w| as its mantissa: the value w * 2^-133, exactly (bf16 numbers
+// with a zero exponent field are the multiples of 2^-133 below 2^-126).  Products with such an operand are
 // 2^133 times too small, so the other operand, the routed rows and H, is kept at kActScale times
 // its value, which holds the fp32 accumulator above its own subnormal range for activations down
 // to about 1e-20; the epilogues multiply the scales by kAccScaleChannel.  Every step is an exact

@@ -1,23 +1,33 @@
 // pack.cu -- one-time weight layout change for the TMEM-operand GEMMs: every expert's
 // int8 matrix stored [in, out] (x @ W orientation) becomes [out, in], so that the
-// reduction elements of one output feature are contiguous, and each value w is stored in
-// sign-magnitude form (bit 7 the sign, bits 0..6 |w|), which the GEMMs' converters turn
-// into a bf16 operand in two instructions per pair of values (kActScale in kernels.cuh).
-// -128 has no such form: it is reported through `range_flag`.  Scales are untouched (they
-// stay per output channel).
+// reduction elements of one output feature are contiguous, and every four consecutive
+// values w[k..k+3] become one 32-bit word of sign bits and 7-bit magnitudes with the signs
+// crossed over within each 16-bit half (the layout gemm_common.cuh's pk_lo / pk_hi read:
+// bytes sign(w[k+2]) | |w[k]|, sign(w[k]) | |w[k+2]|, sign(w[k+3]) | |w[k+1]|,
+// sign(w[k+1]) | |w[k+3]|), which the GEMMs' converters turn into bf16 operands in three
+// instructions per four values (kActScale in kernels.cuh).  -128 has no such form: it is
+// reported through `range_flag`.  Scales are untouched (they stay per output channel).
 #include "kernels.cuh"
 
 namespace moe {
 
 namespace {
 
-// a two's-complement byte -> its sign-magnitude byte (-128 -> 0x80, flagged by the caller)
-__device__ __forceinline__ uint32_t sign_magnitude(uint32_t b)
+// four two's-complement bytes w[k..k+3] (byte i of `w4` = w[k+i]) -> the packed word
+__device__ __forceinline__ uint32_t pack_word(uint32_t w4)
 {
-    return (b & 0x80u) ? (0x80u | ((0x100u - b) & 0x7Fu)) : b;
+    uint32_t mag[4], sgn[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t b = (w4 >> (8 * i)) & 0xFFu;
+        sgn[i] = b >> 7;
+        mag[i] = (sgn[i] ? 0x100u - b : b) & 0x7Fu;   // -128 gives 0: flagged by the caller
+    }
+    return (mag[0] | sgn[2] << 7) | (mag[2] | sgn[0] << 7) << 8 | (mag[1] | sgn[3] << 7) << 16 |
+           (mag[3] | sgn[1] << 7) << 24;
 }
 
-// 64 x 64-byte tiles through shared memory: out[e, m, k] = sm(in[e, k, m])
+// 64 x 64-byte tiles through shared memory: out[e, m, k] = in[e, k, m], four k at a time packed
 __global__ void __launch_bounds__(256) pack_i8_kernel(const int8_t *in, int8_t *out, int K, int M, int *range_flag)
 {
     __shared__ uint32_t tile[64][17];   // [k][m / 4], padded
@@ -39,9 +49,9 @@ __global__ void __launch_bounds__(256) pack_i8_kernel(const int8_t *in, int8_t *
         for (int b = 0; b < 4; ++b) {
             const uint32_t byte = (tile[ks + q * 4 + b][mm >> 2] >> (8 * (mm & 3))) & 0xffu;
             minus128 |= byte == 0x80u;
-            acc |= sign_magnitude(byte) << (8 * b);
+            acc |= byte << (8 * b);
         }
-        w[q] = acc;
+        w[q] = pack_word(acc);
     }
     *reinterpret_cast<uint4 *>(out + (static_cast<size_t>(e) * M + m0 + mm) * K + k0 + ks) =
         make_uint4(w[0], w[1], w[2], w[3]);

@@ -350,15 +350,22 @@ def test_cta_pairs_match_single_cta(m, tiny_inputs, tiny_handle, T, mode):
     parity.check_output(paired, tiny_inputs.layers[0], tiny_inputs.x[:T], range(T), near)
 
 
-def _sign_magnitude(w):
-    """The packed byte of each int8 value: bit 7 the sign, bits 0..6 the magnitude."""
-    wi = w.to(torch.int16)
-    return torch.where(wi < 0, 0x80 | (-wi), wi).to(torch.uint8)
+def _packed_bytes(wt):
+    """The packed bytes of int8 values wt [..., K] (K contiguous, the input elements of one output
+    feature): every four values w0..w3 become the bytes s2|m0, s0|m2, s3|m1, s1|m3, where mi = |wi|
+    and si = 0x80 for a negative wi."""
+    wi = wt.to(torch.int16).reshape(*wt.shape[:-1], -1, 4)
+    m = wi.abs()
+    sg = (wi < 0).to(torch.int16) * 0x80
+    out = torch.stack([sg[..., 2] | m[..., 0], sg[..., 0] | m[..., 2], sg[..., 3] | m[..., 1], sg[..., 1] | m[..., 3]],
+                      dim=-1)
+    return out.reshape(wt.shape).to(torch.uint8)
 
 
 def test_pack_weight_layout(m, tiny_handle):
-    """moe_pack_weight transposes each expert and stores every value of [-127, 127] in
-    sign-magnitude form; a tensor holding -128 is refused with MOE_ERANGE."""
+    """moe_pack_weight transposes each expert and stores every value of [-127, 127] as a sign and a
+    magnitude, four values to a word with crossed signs; a tensor holding -128 is refused with
+    MOE_ERANGE."""
     h, _, _ = tiny_handle
     g = torch.Generator(device="cuda").manual_seed(3)
     for which, shape in ((0, (8, 256, 512)), (1, (8, 512, 256))):
@@ -366,13 +373,13 @@ def test_pack_weight_layout(m, tiny_handle):
         p = torch.empty((shape[0], shape[2], shape[1]), dtype=torch.int8, device="cuda")
         m.check(m.moe_pack_weight(h, w, p, which))
         torch.cuda.synchronize()
-        assert torch.equal(p.view(torch.uint8), _sign_magnitude(w.transpose(1, 2)))
+        assert torch.equal(p.view(torch.uint8), _packed_bytes(w.transpose(1, 2)))
         # a rank's share of the experts: exactly its bytes are read and written
         part = w[2:5].contiguous()
         guard = torch.full((4, shape[2], shape[1]), 7, dtype=torch.int8, device="cuda")
         m.check(m.moe_pack_weight_n(h, part, guard, which, 3))
         torch.cuda.synchronize()
-        assert torch.equal(guard[:3].view(torch.uint8), _sign_magnitude(part.transpose(1, 2)))
+        assert torch.equal(guard[:3].view(torch.uint8), _packed_bytes(part.transpose(1, 2)))
         assert bool((guard[3] == 7).all())
         # one -128 anywhere: no packed form
         w.view(-1)[12345] = -128
