@@ -40,7 +40,8 @@ def test_library_needs_no_cuda_shared_library(m):
 
 def test_strerror_and_version(m):
     assert m.moe_strerror(0) == "ok"
-    for code in (m.MOE_EINVAL, m.MOE_EUNSUPPORTED, m.MOE_ENOMEM, m.MOE_ECUDA, m.MOE_ETIMEOUT, m.MOE_ENODEV):
+    for code in (m.MOE_EINVAL, m.MOE_EUNSUPPORTED, m.MOE_ENOMEM, m.MOE_ECUDA, m.MOE_ETIMEOUT, m.MOE_ENODEV,
+                 m.MOE_ERANGE):
         assert m.moe_strerror(code) not in ("ok", "unknown status code")
     assert m.moe_strerror(12345) == "unknown status code"
     assert m.moe_version() >= 100
