@@ -442,18 +442,32 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
         api = "moe_forward_host (moe_set_host_overlap on)"
     for _ in range(max(1, W // 2)):
         e2e_step()
+    # timed like the device figure: R regions of K steps, the median region, so that both run for
+    # about as long under the same power cap
+    e2e_clocks = ClockSampler(dev.index) if rank == 0 else None
+    if e2e_clocks:
+        e2e_clocks.start()
+    e2e_regions = []
+    for r in range(R):
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        if e2e_clocks and r == 0:
+            e2e_clocks.mark("t0")
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_regions.append(e0.elapsed_time(e1))
+    if e2e_clocks:
+        e2e_clocks.mark("t1")
     barrier(world, dev)
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(K):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, world, dev)
+    e2e_clk = e2e_clocks.stop() if e2e_clocks else None
+    e2e_ms = max_over_ranks(statistics.median(e2e_regions) / K, world, dev)
     moe.check(moe.moe_sync_status(h.h, stream))
     nb = T * w.d * 2
     rec["e2e"] = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": nb,
-                  "d2h_bytes_per_step": nb, "ms_per_step": e2e_ms, "api": api}
+                  "d2h_bytes_per_step": nb, "ms_per_step": e2e_ms, "repeats": R, "api": api, "clocks": e2e_clk}
 
     peaks, peak_src = measured_peaks()
     work = algorithmic_work(w, T, n_touched, counts, args.scale_block)
