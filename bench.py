@@ -16,7 +16,10 @@ layout's decode and prefill, each measured the same way.
 
 Timing: W untimed warm-up steps, then R repeats of a region of exactly K steps,
 each bracketed by a barrier and a device synchronisation and timed with CUDA events
-on the launching stream; the reported time is the median region.  Inputs are
+on the launching stream; the reported time is the median region.  After each timed
+region the same K steps run again with events around every launch: the per-kernel
+durations (the median over those regions) behind the roofline come from the same clock
+and power-cap conditions as the timed regions, which carry no events.  Inputs are
 resident in HBM when a region starts; the layer weights (4.8 GB per layer) are
 larger than L2, so every step streams them from HBM.  Under torchrun each rank runs
 an independent replica on its own GPU and its own token batch (no collective on the
@@ -359,11 +362,16 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
     R = repeats_for(e0.elapsed_time(e1) / W, K, args.repeats)
     R = int(max_over_ranks(R, world, dev))   # every rank runs the same number of regions
 
-    # R regions of exactly K steps, device-timed; the median region is reported
+    # R regions of exactly K steps, device-timed; the median region is reported.  Unless the extras
+    # are skipped, each timed region is followed by the same K steps with events around every launch
+    # (moe_set_profiling), so that the per-kernel durations behind the roofline come from the same
+    # clock and power-cap conditions as the timed regions; the timed regions themselves carry no
+    # events.
     clocks = ClockSampler(dev.index) if rank == 0 else None
     if clocks:
         clocks.start()
     region_ms = []
+    kernel_regions = []   # per profiled region: {kernel: (total ms, launches)}
     for r in range(R):
         barrier(world, dev)
         torch.cuda.synchronize(dev)
@@ -375,6 +383,16 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         region_ms.append(e0.elapsed_time(e1))
+        if not args.skip_extras:
+            moe.check(moe.moe_set_profiling(h.h, True))
+            moe.moe_get_kernel_times(h.h)
+            for _ in range(K):
+                step()
+            torch.cuda.synchronize(dev)
+            rc, kt = moe.moe_get_kernel_times(h.h)
+            moe.check(rc)
+            moe.check(moe.moe_set_profiling(h.h, False))
+            kernel_regions.append(kt)
     if clocks:
         clocks.mark("t1")
     barrier(world, dev)
@@ -402,18 +420,10 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
         rec["note"] = "profiling variant: no per-kernel or end-to-end pass"
         return rec, None
 
-    # per-kernel durations: K more steps with events around every launch
-    moe.check(moe.moe_set_profiling(h.h, True))
-    moe.moe_get_kernel_times(h.h)
-    barrier(world, dev)
-    for _ in range(K):
-        step()
-    torch.cuda.synchronize(dev)
-    rc, ktimes = moe.moe_get_kernel_times(h.h)
-    moe.check(rc)
-    moe.check(moe.moe_set_profiling(h.h, False))
-    per_launch = {k: (t / n if n else 0.0) for k, (t, n) in ktimes.items()}
-    launches_per_step = sum(n for _, n in ktimes.values()) / K
+    # per-kernel durations: the median over the profiled regions of each kernel's mean launch time
+    per_launch = {k: statistics.median([(kt[k][0] / kt[k][1] if kt[k][1] else 0.0) for kt in kernel_regions])
+                  for k in kernel_regions[0]}
+    launches_per_step = sum(n for _, n in kernel_regions[0].values()) / K
 
     # routing of the last step -> experts that received tokens
     offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
@@ -440,6 +450,9 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
         def e2e_step():
             moe.check(moe.moe_forward_host(h.h, T, x_host, *moe.layer_args(layers[0]), out_host, stream))
         api = "moe_forward_host (moe_set_host_overlap on)"
+    # the region ends once the last result has reached host memory (the output copies of
+    # host-overlap forwards run on a stream of the handle)
+    e2e_end = (lambda: None) if w.blocks else (lambda: moe.check(moe.moe_host_wait(h.h, stream)))
     for _ in range(max(1, W // 2)):
         e2e_step()
     # timed like the device figure: R regions of K steps, the median region, so that both run for
@@ -456,6 +469,7 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
         e0.record(stream)
         for _ in range(K):
             e2e_step()
+        e2e_end()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_regions.append(e0.elapsed_time(e1))

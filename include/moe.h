@@ -159,7 +159,8 @@ MOE_API int moe_forward(moe_handle h, int T, const void *x, const float *router_
  * (bf16 [T, d]) to the device, runs the layer, copies the result into out_host
  * (bf16 [T, d]), all enqueued on `stream`.  The weights are device pointers.
  * Pinned host buffers make the copies asynchronous; the caller must
- * synchronise the stream (e.g. moe_sync_status) before reading out_host.
+ * synchronise (moe_sync_status) before reading out_host.  With host overlap on
+ * (moe_set_host_overlap) the output copy runs on a stream of the handle.
  */
 MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const float *router_w,
                              const int8_t *w_lin, const void *s_lin, const int8_t *w_v,
@@ -169,16 +170,27 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
 /*
  * Host overlap for moe_forward_host (on = 1; 0, the default, turns it off).  With
  * it on, successive host-buffer forwards of this handle alternate between two
- * device staging slots, and each call copies x_host in on a copy stream of the
- * handle, so the copy overlaps the previous call's layer; the layer and the copy
- * of the result into out_host stay on `stream`.  The input copy waits for its
- * slot's previous call and, where x_host overlaps the host output of the call
+ * device staging slots; each call copies x_host in on one copy stream of the
+ * handle and the result out to out_host on another, so both copies overlap the
+ * neighbouring calls' layers, which stay on `stream`.  The input copy waits for
+ * its slot's previous call and, where x_host overlaps the host output of the call
  * before, for that output (layers chained through host memory), but not for other
  * work enqueued earlier on `stream`: x_host must hold its values when the call is
- * made.  Results are identical with overlap on or off.  Costs a second pair of
- * [T, d] staging buffers.  Returns MOE_EINVAL for a NULL handle or another value.
+ * made.  The output copy follows the call's layer but `stream` does not wait for
+ * it: out_host holds the result after moe_sync_status (which also waits for the
+ * handle's copy streams) or once `stream` has passed moe_host_wait.  Results are
+ * identical with overlap on or off.  Costs a second pair of [T, d] staging
+ * buffers.  Returns MOE_EINVAL for a NULL handle or another value.
  */
 MOE_API int moe_set_host_overlap(moe_handle h, int on);
+
+/*
+ * Make `stream` wait (on the device, without blocking the host) until every host
+ * copy of the handle's host-overlap forwards issued so far has completed, so that
+ * work or an event enqueued on `stream` afterwards follows the results' arrival in
+ * host memory.  MOE_EINVAL for a NULL handle.
+ */
+MOE_API int moe_host_wait(moe_handle h, void *stream);
 
 /*
  * One residual MoE block ("Transformer stack and language model head": pre/post

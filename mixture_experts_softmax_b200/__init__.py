@@ -42,7 +42,7 @@ EXPORTS = (
     "moe_sync_status", "moe_set_timeout", "moe_set_profiling", "moe_get_kernel_times", "moe_plan",
     "moe_set_weight_layout", "moe_pack_weight", "moe_route_noalloc",
     "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_set_cta_pairs", "moe_pack_weight_n",
-    "moe_set_host_overlap",
+    "moe_set_host_overlap", "moe_host_wait",
 )
 
 
@@ -86,6 +86,7 @@ def _load() -> ctypes.CDLL:
         "moe_ep_combine": (I, [P, I, P, P, P]),
         "moe_set_cta_pairs": (I, [P, I]),
         "moe_set_host_overlap": (I, [P, I]),
+        "moe_host_wait": (I, [P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -218,6 +219,10 @@ def moe_set_cta_pairs(h, mode: int) -> int:
 
 def moe_set_host_overlap(h, on: int) -> int:
     return _lib.moe_set_host_overlap(h, int(on))
+
+
+def moe_host_wait(h, stream=None) -> int:
+    return _lib.moe_host_wait(h, _stream(stream))
 
 
 def moe_set_weight_layout(h, layout: int) -> int:

@@ -56,12 +56,14 @@ struct moe_ctx {
     DevBuf b_part;     // fp32 [num_sms, 128, 256]: the GEMMs' last-wave partial sums
     // host-buffer forwards with host overlap on (moe_set_host_overlap): two staging slots, each
     // x [T, d] then out [T, d] bf16, used by alternate calls.  A call copies its input in on
-    // copy_in, so it can overlap the previous call's layer on the caller's stream.
+    // copy_in and its result out on copy_out, so both copies overlap the neighbouring calls'
+    // layers on the caller's stream.
     bool host_overlap = false;
     DevBuf b_host[2];
     int host_slot = 0;
-    cudaStream_t copy_in = nullptr;
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
     cudaEvent_t ev_in[2] = {nullptr, nullptr};     // slot k's input has landed
+    cudaEvent_t ev_layer[2] = {nullptr, nullptr};  // slot k's layer has written its result
     cudaEvent_t ev_done[2] = {nullptr, nullptr};   // slot k's last call has copied its output out
     bool slot_used[2] = {false, false};
     const char *slot_out[2] = {nullptr, nullptr};  // the host output range of slot k's last call
@@ -199,6 +201,7 @@ RouteLayout route_layout(int T, int E)
 int sync_last(moe_ctx *h)
 {
     if (h->copy_in && cudaStreamSynchronize(h->copy_in) != cudaSuccess) return MOE_ECUDA;
+    if (h->copy_out && cudaStreamSynchronize(h->copy_out) != cudaSuccess) return MOE_ECUDA;
     if (!h->used) return MOE_OK;
     return cudaStreamSynchronize(h->last_stream) == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
@@ -796,9 +799,11 @@ MOE_API int moe_destroy(moe_handle h)
         if (b->ptr) cudaFree(b->ptr);
     for (int k = 0; k < 2; ++k) {
         if (h->ev_in[k]) cudaEventDestroy(h->ev_in[k]);
+        if (h->ev_layer[k]) cudaEventDestroy(h->ev_layer[k]);
         if (h->ev_done[k]) cudaEventDestroy(h->ev_done[k]);
     }
     if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
     if (h->err) cudaFree(h->err);
     if (h->b_part.ptr) cudaFree(h->b_part.ptr);
     for (auto &p : h->pending) {
@@ -920,6 +925,10 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
     if ((rc = begin_call(h, T, s)) != MOE_OK) return rc;
     const size_t xb = static_cast<size_t>(T) * h->d * 2;
     if (!h->host_overlap) {
+        // output copies of earlier overlapped calls may still be running on copy_out: land them first
+        // (this call may write the same host buffer)
+        for (int k = 0; k < 2; ++k)
+            if (h->slot_used[k] && cudaStreamWaitEvent(s, h->ev_done[k], 0) != cudaSuccess) return MOE_ECUDA;
         char *xs = static_cast<char *>(h->b_stage.ptr);
         char *os = xs + xb;
         if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ECUDA;
@@ -929,11 +938,15 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
         if (cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
         return MOE_OK;
     }
-    // host overlap: slot k alternates between calls; the input copy runs on copy_in
+    // host overlap: slot k alternates between calls; the input copy runs on copy_in, the output
+    // copy on copy_out
     if (!h->copy_in) {
-        if (cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking) != cudaSuccess) return MOE_ECUDA;
+        if (cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking) != cudaSuccess)
+            return MOE_ECUDA;
         for (int j = 0; j < 2; ++j)
             if (cudaEventCreateWithFlags(&h->ev_in[j], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&h->ev_layer[j], cudaEventDisableTiming) != cudaSuccess ||
                 cudaEventCreateWithFlags(&h->ev_done[j], cudaEventDisableTiming) != cudaSuccess)
                 return MOE_ECUDA;
     }
@@ -953,8 +966,12 @@ MOE_API int moe_forward_host(moe_handle h, int T, const void *x_host, const floa
     if ((rc = run_layer(h, T, xs, router_w, w_lin, s_lin, w_v, s_v, w_1, s_1, os, nullptr, nullptr, nullptr, 0.f, s)) !=
         MOE_OK)
         return rc;
-    if (cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaEventRecord(h->ev_done[k], s) != cudaSuccess)
+    // the result goes out on copy_out once the layer has written it; the next call's layer on s does
+    // not wait for it (it uses the other slot), and this slot's next input copy, on which the
+    // layer that reuses the slot waits, waits for it (ev_done)
+    if (cudaEventRecord(h->ev_layer[k], s) != cudaSuccess || cudaStreamWaitEvent(h->copy_out, h->ev_layer[k], 0) != cudaSuccess ||
+        cudaMemcpyAsync(out_host, os, xb, cudaMemcpyDeviceToHost, h->copy_out) != cudaSuccess ||
+        cudaEventRecord(h->ev_done[k], h->copy_out) != cudaSuccess)
         return MOE_ECUDA;
     h->slot_used[k] = true;
     h->slot_out[k] = static_cast<const char *>(out_host);
@@ -967,6 +984,15 @@ MOE_API int moe_set_host_overlap(moe_handle h, int on)
 {
     if (!h || (on != 0 && on != 1)) return MOE_EINVAL;
     h->host_overlap = on != 0;
+    return MOE_OK;
+}
+
+MOE_API int moe_host_wait(moe_handle h, void *stream)
+{
+    if (!h) return MOE_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int k = 0; k < 2; ++k)
+        if (h->slot_used[k] && cudaStreamWaitEvent(s, h->ev_done[k], 0) != cudaSuccess) return MOE_ECUDA;
     return MOE_OK;
 }
 
@@ -1023,6 +1049,9 @@ MOE_API int moe_sync_status(moe_handle h, void *stream)
 {
     if (!h) return MOE_EINVAL;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ECUDA;
+    // host-overlap copies run on the handle's own streams
+    if (h->copy_in && cudaStreamSynchronize(h->copy_in) != cudaSuccess) return MOE_ECUDA;
+    if (h->copy_out && cudaStreamSynchronize(h->copy_out) != cudaSuccess) return MOE_ECUDA;
     if (!h->err) return MOE_OK;
     int e = 0;
     if (cudaMemcpy(&e, h->err, sizeof e, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ECUDA;

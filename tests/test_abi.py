@@ -182,5 +182,8 @@ def test_host_overlap_switch(m):
         assert m.moe_set_host_overlap(h, 0) == m.MOE_OK
         assert m.moe_set_host_overlap(h, 2) == m.MOE_EINVAL
         assert m.moe_set_host_overlap(None, 1) == m.MOE_EINVAL
+        # nothing in flight: nothing to wait for (no CUDA call is made)
+        assert m.moe_host_wait(h, None) == m.MOE_OK
+        assert m.moe_host_wait(None, None) == m.MOE_EINVAL
     finally:
         m.moe_destroy(h)

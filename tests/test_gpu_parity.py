@@ -188,6 +188,43 @@ def test_host_overlap_streams_and_pageable_memory(m, tiny_inputs, tiny_handle):
         assert torch.equal(out, ref)
 
 
+def test_host_wait_orders_the_output_copies(m, tiny_inputs, tiny_handle):
+    """With host overlap on, the output copies run on a stream of the handle: after moe_host_wait on
+    the caller's stream and a synchronisation of that stream alone (no moe_sync_status), every
+    output holds the serial path's result, bit for bit.  A serial call afterwards into the same host
+    buffer lands after the overlapped call's copy."""
+    h, layer, _ = tiny_handle
+    m.check(m.moe_set_router_bias(h, None))
+    m.check(m.moe_set_padding_mask(h, None))
+    T = 300
+    xs = [tiny_inputs.x[i * 8:i * 8 + T].clone().pin_memory() for i in range(4)]
+    refs = []
+    for x in xs:
+        r = torch.empty_like(x).pin_memory()
+        m.check(m.moe_forward_host(h, T, x, *m.layer_args(layer), r))
+        refs.append(r)
+    m.check(m.moe_sync_status(h))
+    st = torch.cuda.Stream()
+    outs = [torch.empty_like(x).pin_memory() for x in xs]
+    try:
+        m.check(m.moe_set_host_overlap(h, 1))
+        for x, out in zip(xs, outs):
+            m.check(m.moe_forward_host(h, T, x, *m.layer_args(layer), out, st))
+        m.check(m.moe_host_wait(h, st))
+        st.synchronize()
+        for out, ref in zip(outs, refs):
+            assert torch.equal(out, ref)
+        # an overlapped call, then a serial one writing the same host buffer: the serial result wins
+        m.check(m.moe_forward_host(h, T, xs[0], *m.layer_args(layer), outs[1], st))
+        m.check(m.moe_set_host_overlap(h, 0))
+        m.check(m.moe_forward_host(h, T, xs[1], *m.layer_args(layer), outs[1], st))
+        m.check(m.moe_sync_status(h, st))
+        assert torch.equal(outs[1], refs[1])
+    finally:
+        m.check(m.moe_set_host_overlap(h, 0))
+        m.check(m.moe_sync_status(h))
+
+
 def test_kernel_times_reported(m, tiny_inputs, tiny_handle):
     h, layer, _ = tiny_handle
     x = tiny_inputs.x[:64].cuda()
