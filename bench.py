@@ -420,10 +420,7 @@ def bench_workload(name, args, world, rank, dev, layout, cpu_seconds, with_cpu):
         rec["note"] = "profiling variant: no per-kernel or end-to-end pass"
         return rec, None
 
-    # per-kernel durations: the median over the profiled regions of each kernel's mean launch time
-    per_launch = {k: statistics.median([(kt[k][0] / kt[k][1] if kt[k][1] else 0.0) for kt in kernel_regions])
-                  for k in kernel_regions[0]}
-    launches_per_step = sum(n for _, n in kernel_regions[0].values()) / K
+    per_launch, launches_per_step = kernel_times_over_regions(kernel_regions, K)
 
     # routing of the last step -> experts that received tokens
     offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
@@ -603,6 +600,17 @@ def run_native(args, world, rank, local):
             subs[key] = sub
         line["workloads"] = subs
     return line
+
+
+def kernel_times_over_regions(kernel_regions, K):
+    """Per kernel, the median over the profiled regions of its mean launch time (ms), and the
+    library's launches per step.  kernel_regions: one {kernel: (total ms, launches)} per region of
+    K steps (moe_get_kernel_times after each region); a kernel that did not run reads 0."""
+    names = list(kernel_regions[0])
+    per_launch = {k: statistics.median([(kt[k][0] / kt[k][1] if kt[k][1] else 0.0) for kt in kernel_regions])
+                  for k in names}
+    launches_per_step = sum(n for _, n in kernel_regions[0].values()) / K
+    return per_launch, launches_per_step
 
 
 def cpu_baseline(w, cpu_layers, inp, budget_s):

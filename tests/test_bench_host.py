@@ -60,3 +60,19 @@ def test_recorded_traffic_is_keyed(tmp_path, monkeypatch):
 def test_source_hash_covers_each_layouts_gemm():
     assert bench.kernel_source_hash("packed") != bench.kernel_source_hash("in_out")
     assert set(bench.GEMM_SOURCES["packed"]) >= {"gemm_ts.cu", "gemm_common.cuh", "ptx.cuh"}
+
+
+def test_kernel_times_over_regions():
+    """The per-kernel times behind the roofline: each kernel's mean launch time per profiled region,
+    then the median over the regions (so one region under a different clock does not move it);
+    kernels that did not run read 0; launches per step from the region's launch counts."""
+    K = 10
+    regions = [
+        {"up_proj": (100.0, 10), "down_proj": (50.0, 10), "router": (0.0, 0)},
+        {"up_proj": (130.0, 10), "down_proj": (52.0, 10), "router": (0.0, 0)},   # a slow region
+        {"up_proj": (101.0, 10), "down_proj": (51.0, 10), "router": (0.0, 0)},
+    ]
+    per_launch, lps = bench.kernel_times_over_regions(regions, K)
+    assert per_launch == {"up_proj": 10.1, "down_proj": 5.1, "router": 0.0}
+    assert lps == 2.0
+
