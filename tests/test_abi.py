@@ -25,6 +25,48 @@ def test_header_declares_the_binding_exports(m):
     assert declared_symbols() == sorted(m.EXPORTS)
 
 
+def declared_parameters():
+    """name -> the kinds of its parameters in include/moe.h: 'p' pointer (moe_handle included), 'i' int
+    (int, int32_t), 'f' float, 'l' long long."""
+    src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "moe.h")).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(([^)]*)\)", src):
+        kinds = []
+        for prm in (q.strip() for q in params.split(",")):
+            if prm in ("", "void"):
+                continue
+            if "*" in prm or prm.startswith("moe_handle"):
+                kinds.append("p")
+            elif prm.startswith("long long"):
+                kinds.append("l")
+            elif prm.startswith("float"):
+                kinds.append("f")
+            else:
+                assert prm.split()[0] in ("int", "int32_t"), prm
+                kinds.append("i")
+        out[name] = kinds
+    return out
+
+
+def test_binding_signatures_follow_the_header(m):
+    """Every ctypes signature the binding sets has the header's parameter count and kinds, so a call
+    through the binding passes each argument in the width the library reads."""
+    def kind(t):
+        if t is ctypes.c_int:
+            return "i"
+        if t is ctypes.c_float:
+            return "f"
+        if t is ctypes.c_longlong:
+            return "l"
+        return "p"   # c_void_p and POINTER(...)
+    lib = m.lib()
+    declared = declared_parameters()
+    assert sorted(declared) == sorted(m.EXPORTS)
+    for name, kinds in declared.items():
+        got = [kind(t) for t in getattr(lib, name).argtypes]
+        assert got == kinds, (name, got, kinds)
+
+
 def test_library_exports_every_declared_symbol(m):
     lib = ctypes.CDLL(m.LIB_PATH)
     for name in declared_symbols():
