@@ -109,6 +109,13 @@ constexpr int kCtlTickets = 64;     // first GEMM ticket
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// the packed layout's power-of-two steps must undo each other exactly: weights enter the tensor
+// cores at 2^-133 times their value, activations at kActScale times theirs
+static_assert(static_cast<double>(kAccScaleChannel) * static_cast<double>(kActScale) == 0x1p133,
+              "per-channel epilogue factor must be 2^133 / kActScale");
+static_assert(static_cast<double>(kActUnscale) * static_cast<double>(kActScale) == 1.0,
+              "kActUnscale must be the inverse of kActScale");
+
 // the GEMM epilogues' factor from an accumulator to its value: the packed layout's operands are
 // scaled (kActScale); the shared-memory kernels of the [E, in, out] layout ignore it
 float acc_factor(const moe_ctx *h)
